@@ -1,0 +1,240 @@
+"""Integer W8A8 pipeline of the SSD scan (persistent INT8 state) — TEST INFRASTRUCTURE ONLY.
+
+Follows "SSDi8: Accurate and Efficient 8-bit Quantization for State Space
+Duality" (ICLR 2026 paper notes):
+* key design 3: B and C are quantised once, along the group axis G, at SSD entry;
+* key design 1, eq. 4 and the reconstruction: State_INT32 = Q(X_scaled) × Q(B)
+  with X_scaled = LUT_state ⊙ X, LUT_state = Δ ⊙ Decay_state, X_scaled quantised
+  per (H,P);
+* key design 2: State_INT32 requantised to INT8 in registers with per-(H,P)
+  scales (N not quantised), and eq. 6: the inter-chunk decay as a fixed-point
+  code divided by S = 2^k, k = 7, i.e. a multiply and a shift;
+* ChunkBMM and ChunkScan1 reuse the INT8 B and C; ChunkScan2 stays in floating
+  point with the CB dequantisation scale folded into LUT_Scan2.
+
+Readings of points the notes leave open (each also stated in the design notes):
+* quantiser: symmetric, step-size convention q = clamp(rint(v / s), ±127);
+* requantisation: S8 = clamp(rint(acc · (s_x·s_B/s_s)), ±127) — the printed
+  formula's q_max factor is read as part of the step-size scales;
+* eq. 6: H_{c+1} = sat127(S8_c + ((dq_c·H_c + 2^(k-1)) >> k)), dq_c =
+  rint(exp(Acs_last)·2^k) ∈ [0, 2^k]; the shift is arithmetic, so the rounding is
+  half-up; the sum is formed in int32 and then saturated;
+* everything that decides an integer is computed in float32, op by op, in the
+  order written here (IEEE round-to-nearest-even, no fused multiply-add):
+  - ChunkCumsum order: lane l of 32 holds elements [l·m, (l+1)·m), m = Q/32;
+    sequential inclusive sum inside the lane; Kogge-Stone inclusive scan of
+    the lane totals (offsets 1, 2, 4, 8, 16); the exclusive lane prefix
+    (0 for lane 0) is added to each local inclusive sum;
+  - exp is `exp_f32` below (Cody-Waite range reduction, degree-7 Taylor
+    polynomial by Horner, each product and sum rounded separately);
+  - reciprocals of scales are IEEE divisions 1/s.
+
+Parity: every integer (Bq, Cq, Xq, the INT32 accumulators, S8, H8, dq) and the
+float32 Acs are reproducible bit for bit.  Pinned by the exact-representable
+case (A = 0, dyadic inputs: the pipeline must equal the fp64 definition
+exactly), the integer-range and saturation tests, the A = 0 prefix-sum form of
+the recursion, and exp_f32's error bound against fp64 exp.  The rounding modes
+(half-even for rint, half-up for the shift) are this library's specification:
+parity unpinned by the notes, which do not state them.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+QMAX = 127
+F32 = np.float32
+
+# Cody-Waite split of ln 2: the high part is ln 2 rounded to 11 significant bits
+# (1420/2048), so k·LN2_HI is exact for |k| < 2^13; the low part is the rest.
+_LOG2E = F32(1.4426950408889634)
+_LN2_HI = F32(1420.0 / 2048.0)
+_LN2_LO = F32(0.6931471805599453 - 1420.0 / 2048.0)
+# Taylor coefficients 1/n!, n = 0..7, rounded to float32.
+_TAYLOR = [F32(1.0), F32(1.0), F32(0.5), F32(1.0 / 6.0), F32(1.0 / 24.0), F32(1.0 / 120.0),
+           F32(1.0 / 720.0), F32(1.0 / 5040.0)]
+EXP_LO = F32(-87.0)
+EXP_HI = F32(88.0)
+
+
+def exp_f32(x) -> np.ndarray:
+    """exp in float32 with a fixed sequence of rounded operations.
+
+    x < -87 gives 0; x is clamped to at most 88.  k = rint(x·log2e);
+    r = (x − k·ln2_hi) − k·ln2_lo; p = Σ_{n≤7} r^n/n! by Horner; result p·2^k.
+    exp_f32(0) = 1 exactly.
+    """
+    x = np.asarray(x, dtype=F32)
+    xc = np.clip(x, EXP_LO - F32(1.0), EXP_HI)      # below -87 the result is 0 anyway
+    k = np.rint(xc * _LOG2E)
+    r = (xc - k * _LN2_HI) - k * _LN2_LO
+    p = _TAYLOR[7]
+    for n in range(6, -1, -1):
+        p = p * r + _TAYLOR[n]
+    ki = np.clip(k, -126, 127).astype(np.int32)
+    two_k = np.ldexp(F32(1.0), ki).astype(F32)
+    out = (p * two_k).astype(F32)
+    return np.where(x < EXP_LO, F32(0.0), out).astype(F32)
+
+
+def chunk_cumsum_f32(a: np.ndarray) -> np.ndarray:
+    """Inclusive cumulative sum over the last axis (length Q, a multiple of 32), float32,
+    in the 32-lane order described in the module docstring."""
+    a = np.asarray(a, dtype=F32)
+    Q = a.shape[-1]
+    m = Q // 32
+    lanes = a.reshape(a.shape[:-1] + (32, m))
+    s = np.empty_like(lanes)
+    s[..., 0] = lanes[..., 0]
+    for i in range(1, m):
+        s[..., i] = s[..., i - 1] + lanes[..., i]
+    v = s[..., m - 1].copy()
+    lane = np.arange(32)
+    for off in (1, 2, 4, 8, 16):
+        u = np.zeros_like(v)
+        u[..., off:] = v[..., :-off]
+        v = np.where(lane >= off, u + v, v).astype(F32)
+    excl = np.zeros_like(v)
+    excl[..., 1:] = v[..., :-1]
+    return (excl[..., None] + s).reshape(a.shape).astype(F32)
+
+
+def quantize_sym(v: np.ndarray, inv_scale) -> np.ndarray:
+    """clamp(rint(v · inv_scale), ±127) in float32, as int8."""
+    q = np.rint(np.asarray(v, F32) * np.asarray(inv_scale, F32))
+    return np.clip(q, -QMAX, QMAX).astype(np.int8)
+
+
+def quantize_inputs(B_vals: np.ndarray, C_vals: np.ndarray, s_B, s_C):
+    """B and C (float32 values of the bf16 inputs, [Bt,L,G,N]) → int8 with per-G scales."""
+    inv_B = F32(1.0) / np.asarray(s_B, F32)
+    inv_C = F32(1.0) / np.asarray(s_C, F32)
+    Bq = quantize_sym(B_vals, inv_B[None, None, :, None])
+    Cq = quantize_sym(C_vals, inv_C[None, None, :, None])
+    return Bq, Cq
+
+
+def _imatmul(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Exact integer matmul (int64) with a check that the result fits int32."""
+    r = np.matmul(a.astype(np.int64), b.astype(np.int64))
+    assert np.abs(r).max(initial=0) < 2 ** 31, "int32 accumulator overflow"
+    return r
+
+
+def state_passing_i8(S8: np.ndarray, dq: np.ndarray, k: int = 7) -> np.ndarray:
+    """StatePassing on INT8 states (eq. 6 with S = 2^k), sequential over chunks.
+
+    S8 int8 [Bt,nc,H,P,N]; dq int [Bt,H,nc] (decay codes rint(d·2^k)).
+    H_0 = 0;  H_{c+1} = clamp(S8_c + ((dq_c·H_c + 2^(k-1)) >> k), ±127), int32 arithmetic.
+    Returns int8 [Bt,nc+1,H,P,N]; entry c is the state entering chunk c, entry nc the final one.
+    """
+    Bt, nc, H, P, N = S8.shape
+    out = np.zeros((Bt, nc + 1, H, P, N), dtype=np.int8)
+    half = np.int32(1 << (k - 1))
+    dq = np.asarray(dq, np.int32)
+    for c in range(nc):
+        carried = (dq[:, :, c, None, None] * out[:, c].astype(np.int32) + half) >> np.int32(k)
+        out[:, c + 1] = np.clip(S8[:, c].astype(np.int32) + carried, -QMAX, QMAX).astype(np.int8)
+    return out
+
+
+def ssd_w8a8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, chunk: int, k: int = 7) -> dict:
+    """The W8A8 SSD forward.
+
+    x_vals : float32 values of the bf16 x, [Bt,L,H,P]
+    dt [Bt,L,H], A [H], D [H] : float32
+    Bq, Cq : int8 [Bt,L,G,N]
+    s_B, s_C : [G]; s_x, s_s : [H*P] (float32 step sizes)
+    Returns a dict with
+      y      float64 [Bt,L,H,P]  dequantised output (ChunkScan2 and the D skip in fp64)
+      final8 int8 [Bt,H,P,N]     INT8 state after the last token (real value final8·s_s)
+      final  float64 [Bt,H,P,N]  final8 dequantised
+      Acs f32 [Bt,H,nc,Q], dq int32 [Bt,H,nc], Xq int8 [Bt,nc·Q,H,P],
+      acc_state int32 [Bt,nc,H,P,N], S8 int8 [Bt,nc,H,P,N],
+      H8 int8 [Bt,nc,H,P,N] (state entering chunk c), CB int32 [Bt,nc,G,Q,Q],
+      acc_scan1 int32 [Bt,nc·Q,H,P].
+    A final partial chunk is padded with dt = 0, x = 0, Bq = Cq = 0 tokens.
+    """
+    x_vals = np.asarray(x_vals, F32)
+    dt = np.asarray(dt, F32)
+    A = np.asarray(A, F32)
+    D = np.asarray(D, F32)
+    Bt, L, H, P = x_vals.shape
+    G, N = Bq.shape[2], Bq.shape[3]
+    hpg = H // G
+    Q = int(chunk)
+    nc = (L + Q - 1) // Q
+    Lp = nc * Q
+    s_B = np.asarray(s_B, F32)
+    s_C = np.asarray(s_C, F32)
+    s_x = np.asarray(s_x, F32).reshape(H, P)
+    s_s = np.asarray(s_s, F32).reshape(H, P)
+    gh = np.arange(H) // hpg
+
+    def pad(a):
+        w = [(0, 0)] * a.ndim
+        w[1] = (0, Lp - L)
+        return np.pad(a, w)
+
+    xp = pad(x_vals)                                       # [Bt,Lp,H,P]
+    dtp = pad(dt)                                          # [Bt,Lp,H]
+    Bqp = pad(Bq).reshape(Bt, nc, Q, G, N)
+    Cqp = pad(Cq).reshape(Bt, nc, Q, G, N)
+
+    # ChunkCumsum (float32, specified order)
+    a = (dtp * A[None, None, :]).astype(F32)                            # dt·A
+    a_h = np.ascontiguousarray(np.moveaxis(a.reshape(Bt, nc, Q, H), 3, 1))   # [Bt,H,nc,Q]
+    Acs = chunk_cumsum_f32(a_h)
+    last = Acs[..., Q - 1:Q]                                            # [Bt,H,nc,1]
+
+    # ChunkState with the decay moved onto x, quantised per (H,P)
+    dt_h = np.ascontiguousarray(np.moveaxis(dtp.reshape(Bt, nc, Q, H), 3, 1))  # [Bt,H,nc,Q]
+    lut_state = (dt_h * exp_f32((last - Acs).astype(F32))).astype(F32)  # [Bt,H,nc,Q]
+    lut_t = np.moveaxis(lut_state, 1, 3).reshape(Bt, Lp, H)             # back to token-major
+    Xs = (lut_t[..., None] * xp).astype(F32)                            # [Bt,Lp,H,P]
+    inv_sx = (F32(1.0) / s_x).astype(F32)
+    Xq = quantize_sym(Xs, inv_sx[None, None])                           # [Bt,Lp,H,P]
+    Xq_c = Xq.reshape(Bt, nc, Q, H, P)
+    Bq_h = Bqp[:, :, :, gh, :]                                          # [Bt,nc,Q,H,N]
+    acc_state = _imatmul(np.moveaxis(Xq_c, 2, 4),                       # [Bt,nc,H,P,Q]
+                         np.moveaxis(Bq_h, 2, 3))                       # [Bt,nc,H,Q,N]
+    M = ((s_x * s_B[gh][:, None]).astype(F32) / s_s).astype(F32)        # [H,P]
+    S8 = np.clip(np.rint(acc_state.astype(F32) * M[None, None, :, :, None]), -QMAX, QMAX).astype(np.int8)
+
+    # StatePassing: fixed-point decay, multiply and shift
+    dq = np.rint(exp_f32(last[..., 0]) * F32(2 ** k)).astype(np.int32)  # [Bt,H,nc]
+    H8 = state_passing_i8(S8, dq, k)                                    # [Bt,nc+1,H,P,N]
+
+    # ChunkBMM on the INT8 inputs
+    CB = _imatmul(np.moveaxis(Cqp, 3, 2), np.moveaxis(Bqp, 3, 2).swapaxes(-1, -2))   # [Bt,nc,G,Q,Q]
+
+    # ChunkScan1: INT8 C × INT8 state entering the chunk
+    Cq_h = Cqp[:, :, :, gh, :]                                          # [Bt,nc,Q,H,N]
+    acc1 = _imatmul(np.moveaxis(Cq_h, 2, 3),                            # [Bt,nc,H,Q,N]
+                    H8[:, :nc].swapaxes(-1, -2))                        # [Bt,nc,H,N,P]
+    acc_scan1 = np.moveaxis(acc1, 2, 3).reshape(Bt, Lp, H, P)           # [Bt,Lp,H,P]
+
+    # Dequantised output in fp64 from the integer intermediates
+    f64 = np.float64
+    Acs64 = Acs.astype(f64)
+    diff = Acs64[..., :, None] - Acs64[..., None, :]                    # [Bt,H,nc,Q,Q]
+    causal = np.tril(np.ones((Q, Q), dtype=bool))
+    dec = np.where(causal, np.exp(np.where(causal, diff, 0.0)), 0.0)
+    sCB = (s_C.astype(f64) * s_B.astype(f64))[gh]                       # [H]
+    CBh = CB[:, :, gh].astype(f64)                                      # [Bt,nc,H,Q,Q]
+    lut2 = sCB[None, :, None, None, None] * dec * dt_h.astype(f64)[..., None, :]   # [Bt,H,nc,Q,Q]
+    Mmat = CBh * np.moveaxis(lut2, 1, 2)                                # [Bt,nc,H,Q,Q]
+    xc = xp.astype(f64).reshape(Bt, nc, Q, H, P)
+    y_d = np.einsum("bchji,bcihp->bcjhp", Mmat, xc, optimize=True)
+    eA = np.exp(np.moveaxis(Acs64, 1, 3))                               # [Bt,nc,Q,H]
+    y_o = acc1.astype(f64).transpose(0, 1, 3, 2, 4) * (s_C.astype(f64)[gh][:, None]
+                                                       * s_s.astype(f64))[None, None, None] \
+        * eA[..., None]
+    y = (y_d + y_o + D.astype(f64)[None, None, None, :, None] * xc).reshape(Bt, Lp, H, P)[:, :L]
+
+    final8 = H8[:, nc]
+    return {
+        "y": y, "final8": final8, "final": final8.astype(f64) * s_s.astype(f64)[None, :, :, None],
+        "Acs": Acs, "dq": dq, "Xq": Xq, "acc_state": acc_state.astype(np.int32), "S8": S8,
+        "H8": H8[:, :nc], "CB": CB.astype(np.int32), "acc_scan1": acc_scan1.astype(np.int32),
+        "lut_state": lut_state, "M": M,
+    }
