@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Throughput of the SSD chunked scan forward on B200: tokens/s and roofline fraction.
+
+One step = one pass of the whole path over one batch of synthetic input resident in
+HBM: for the W8A8 path ssd_quantize_inputs + ssd_scan_fwd_i8 (ChunkCumsum,
+ChunkState, StatePassing, ChunkBMM/ChunkScan), for the bf16 path ssd_scan_fwd_bf16.
+The default workload is the Mamba-2 2.7B layer shape (B=8, L=8192, H=80, P=64,
+N=128, G=1, chunk 256); its inputs (1.4 GB) are larger than L2, so no flush is
+needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own copy of the workload (independent problems:
+weak scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import multiprocessing as mp
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from harness import WORKLOADS, make_inputs, make_chain, as_float  # noqa: E402
+
+METRIC = "SSD scan fwd tokens/s (B·L/s) and % of roofline, 2.7B layer shape, bf16 & W8A8"
+DATASHEET_HBM_GBS = 8000.0          # the roofline definition's HBM figure (8 TB/s)
+FALLBACK_HBM_GBS = 6650.0           # used only when MEASURED_PEAKS.json is absent
+
+
+# ---------------------------------------------------------------- byte counts
+def path_bytes(w, path: str) -> int:
+    """Compulsory bytes of one step: every input read once, every output written once."""
+    T, H, P, N, G = w.tokens, w.nheads, w.headdim, w.dstate, w.ngroups
+    per_tok = 2 * H * P + 2 * H * P + 4 * G * N + 4 * H      # x, y, B and C (bf16), dt
+    fin = w.batch * H * P * N * (4 if path == "bf16" else 1)
+    params = 8 * H + (0 if path == "bf16" else 4 * (2 * G + 2 * H * P))
+    return T * per_tok + fin + params
+
+
+def kernel_bytes(w, path: str, kernel: str) -> int:
+    """Algorithmic bytes of one launch of `kernel` (its own inputs read once, outputs written once)."""
+    T, H, P, N, G, Q = w.tokens, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
+    nc = w.nchunks
+    chains = w.batch * H
+    states = w.batch * nc * H * P * N
+    bc = 1 if path == "w8a8" else 2                            # bytes per B/C element read by the scan
+    st_w = 1 if path == "w8a8" else 4                           # chunk-state element
+    hc_w = 1 if path == "w8a8" else 2                           # passed-state element
+    acs = chains * nc * Q * 4
+    if kernel == "quantize_inputs":
+        return T * G * N * (2 * 2 + 2 * 1)
+    if kernel == "chunk_cumsum":
+        return T * H * 4 + acs + chains * nc * 4
+    if kernel == "chunk_state":
+        return T * (2 * H * P + bc * G * N + 4 * H) + acs + states * st_w
+    if kernel == "state_passing":
+        return states * st_w + chains * nc * 4 + states * hc_w + w.batch * H * P * N * (4 if path == "bf16" else 1)
+    if kernel == "chunk_scan":
+        return T * (2 * H * P + 2 * bc * G * N + 4 * H + 2 * H * P) + acs + states * hc_w
+    return 0
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
+
+
+# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
+# capture, keyed by kernel name, with the sha1 of the kernel source it was taken on.
+# A kernel whose source changed since reports null.
+NCU_TRAFFIC = {}
+
+
+def _src_hash(kernel: str):
+    f = {"chunk_scan": "chunk_scan.cu", "chunk_state": "chunk_state.cu", "state_passing": "state_passing.cu",
+         "chunk_cumsum": "cumsum.cu", "quantize_inputs": "quantize.cu"}.get(kernel)
+    if not f:
+        return None
+    with open(os.path.join(ROOT, "int8_quant_b200", "csrc", f), "rb") as fh:
+        return hashlib.sha1(fh.read()).hexdigest()
+
+
+def traffic_for(kernel: str, path: str, workload: str):
+    e = NCU_TRAFFIC.get((kernel, path, workload))
+    if not e or e["src_sha1"] != _src_hash(kernel):
+        return None
+    return e["bytes_per_launch"]
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ssd_bench_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+def _oracle_chain(args):
+    """Time the oracle on one (batch, head) chain of the workload (inputs generated untimed)."""
+    name, b, h, path, budget_s = args
+    sys.path.insert(0, ROOT)
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    from harness import WORKLOADS as WL, make_chain as mk, as_float as af
+    from oracle import ssd_fp64 as F, ssd_w8a8 as W
+    w = WL[name]
+    ch = mk(w, b, h)
+    x = af(ch["x"])[None, :, None, :]
+    dt = ch["dt"][None, :, None]
+    Bv = af(ch["B"])[None, :, None, :]
+    Cv = af(ch["C"])[None, :, None, :]
+    A = np.array([ch["A"]], np.float32)
+    D = np.array([ch["D"]], np.float32)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        if path == "bf16":
+            F.ssd_sequential(x, dt, A, Bv, Cv, D)
+        else:
+            sc = F.calibrate(x, dt, A, Bv, Cv, w.chunk, w.calib_prefix)
+            Bq, Cq = W.quantize_inputs(Bv.astype(np.float32), Cv.astype(np.float32), sc["s_B"], sc["s_C"])
+            W.ssd_w8a8(x.astype(np.float32), dt, A, Bq, Cq, D, sc["s_B"], sc["s_C"], sc["s_x"], sc["s_s"],
+                       w.chunk)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            return done, el
+
+
+def cpu_oracle_sample(w, path: str, budget_s: float, pool=None):
+    """Oracle throughput on host cores: each worker repeats one full-length chain for ~budget_s.
+
+    tokens/s = (chains finished × L / H) / slowest worker's time, i.e. the rate at which
+    the oracle would process whole tokens (all H heads)."""
+    cores = os.cpu_count() or 1
+    rs = np.random.default_rng(0)
+    jobs = [(w.name, int(rs.integers(w.batch)), int(rs.integers(w.nheads)), path, budget_s) for _ in range(cores)]
+    own = pool is None
+    if own:
+        pool = mp.get_context("spawn").Pool(cores)
+    try:
+        res = pool.map(_oracle_chain, jobs)
+    finally:
+        if own:
+            pool.close()
+            pool.join()
+    chains = sum(r[0] for r in res)
+    t = max(r[1] for r in res)
+    value = chains * w.seqlen / w.nheads / t
+    sample = (f"{chains} full-length (L={w.seqlen}) (batch, head) chains of {w.name}, "
+              f"{'fp64 sequential recurrence' if path == 'bf16' else 'integer W8A8 pipeline incl. per-chain calibration'}, "
+              f"{cores} spawn workers, {t:.1f} s")
+    return {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args, rank, world, dist):
+    import torch
+    import int8_quant_b200 as iq
+    from int8_quant_b200.runner import SsdProblem, to_device
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    host = make_inputs(w)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        dinp = to_device(host, dev)
+        pb = SsdProblem(dinp, w.chunk, with_i8=True, with_bf16=True)
+        pb.calibrate(w.calib_prefix)            # static W8A8 scales on the prefix (GPU)
+    torch.cuda.synchronize()
+    peak, peak_src = measured_peaks()
+
+    def step_fn(path):
+        if path == "w8a8":
+            return lambda: pb.run_i8(stream)
+        return lambda: pb.run_bf16(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(path):
+        step = step_fn(path)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        iq.ssd_profile_reset()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(dev.index) as clk:
+            barrier()
+            torch.cuda.synchronize()
+            iq.ssd_profile_enable(True)
+            ev0.record(stream)
+            for _ in range(args.steps):
+                step()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            iq.ssd_profile_enable(False)
+            barrier()
+        ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.steps
+        kern = iq.ssd_profile_read()
+        return ms, kern, clk.summary()
+
+    def roofline(path, kern):
+        # dominant kernel = largest share of the step's device time
+        name = max(kern, key=lambda k: kern[k][0])
+        tot_ms, calls = kern[name]
+        per_launch_s = tot_ms / calls / 1e3
+        alg = kernel_bytes(w, path, name)
+        achieved = alg / per_launch_s / 1e9
+        return {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic_for(name, path, w.name),
+                "alg_bytes_per_launch": alg, "launch_ms": round(per_launch_s * 1e3, 4),
+                "peak_source": peak_src,
+                "kernel_shares": {k: round(v[0] / sum(x[0] for x in kern.values()), 4) for k, v in kern.items()}}
+
+    def e2e(path):
+        """Same metric with host buffers: pinned H2D of the step's inputs, the call, D2H of the outputs."""
+        step = step_fn(path)
+        names = ["x", "dt", "B", "C"]
+        hbufs = {k: dinp[k].to("cpu").pin_memory() for k in names}
+        out_dev = [pb.y, pb.final8 if path == "w8a8" else pb.final32]
+        out_host = [torch.empty_like(t, device="cpu").pin_memory() for t in out_dev]
+        h2d = sum(t.numel() * t.element_size() for t in hbufs.values())
+        d2h = sum(t.numel() * t.element_size() for t in out_host)
+        n = max(1, min(args.steps, args.e2e_steps))
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for i in range(n + 1):
+                if i == 1:
+                    barrier()
+                    ev0.record(stream)
+                for k in names:
+                    dinp[k].copy_(hbufs[k], non_blocking=True)
+                step()
+                for dsrc, hdst in zip(out_dev, out_host):
+                    hdst.copy_(dsrc, non_blocking=True)
+            ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = max_over_ranks(ev0.elapsed_time(ev1)) / n
+        return {"value": world * w.tokens / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4), "steps": n}
+
+    results = {}
+    for path in (args.path, "bf16" if args.path == "w8a8" else "w8a8"):
+        ms, kern, clocks = timed(path)
+        launches = sum(c for _, c in kern.values())
+        alg = path_bytes(w, path)
+        results[path] = {
+            "ms_per_step": ms, "value": world * w.tokens / (ms / 1e3), "kern": kern, "clocks": clocks,
+            "roofline": roofline(path, kern), "gpu_launches": launches,
+            "path_roofline": {"alg_bytes": alg, "achieved_GBs": round(alg / (ms / 1e3) / 1e9, 1),
+                              "frac_of_measured_hbm": round(alg / (ms / 1e3) / 1e9 / peak, 4),
+                              "frac_of_8TBs": round(alg / (ms / 1e3) / 1e9 / DATASHEET_HBM_GBS, 4)},
+        }
+        if not args.no_e2e:
+            results[path]["e2e"] = e2e(path)
+    return w, results
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mamba2-2.7b", choices=sorted(WORKLOADS))
+    ap.add_argument("--path", choices=["w8a8", "bf16"], default="w8a8")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work per CPU worker")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    w = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        # The reference arm is the CPU oracle, timed on the host cores; rank 0 only.
+        if rank != 0:
+            return
+        vals = []
+        pool = mp.get_context("spawn").Pool(os.cpu_count() or 1)
+        try:
+            for i in range(args.warmup + args.steps):
+                r = cpu_oracle_sample(w, args.path, args.cpu_budget / 4, pool)
+                if i >= args.warmup:
+                    vals.append(r)
+        finally:
+            pool.close()
+            pool.join()
+        value = statistics.median(v["value"] for v in vals)
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.tokens / value,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64" if args.path == "bf16" else "int64", "data": "synthetic",
+                "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
+                           "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
+                           "path": args.path},
+                "cpu_baseline": {"kind": "oracle", "cores": vals[0]["cores"], "sample": vals[0]["sample"],
+                                 "value": value, "unit": "tokens/s"},
+                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    # CPU pool for the oracle baseline: spawned before the first GPU call.
+    pool = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        pool = mp.get_context("spawn").Pool(os.cpu_count() or 1)
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as td
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = td
+    try:
+        w, res = run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    cpu = None
+    if pool is not None:
+        try:
+            cpu = cpu_oracle_sample(w, args.path, args.cpu_budget, pool)
+        finally:
+            pool.close()
+            pool.join()
+    if rank != 0:
+        return
+    main_r = res[args.path]
+    other = "bf16" if args.path == "w8a8" else "w8a8"
+    o = res[other]
+    line = {
+        "metric": METRIC, "value": main_r["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(main_r["ms_per_step"], 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if args.path == "w8a8" else "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
+                   "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
+                   "path": args.path, "step": ("ssd_quantize_inputs + ssd_scan_fwd_i8" if args.path == "w8a8"
+                                               else "ssd_scan_fwd_bf16"),
+                   "l2": f"inputs larger than L2 ({path_bytes(w, args.path) / 1e9:.2f} GB per step), no flush",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": main_r["roofline"], "path_roofline": main_r["path_roofline"],
+        "cpu_baseline": cpu, "e2e": main_r.get("e2e"), "gpu_launches": main_r["gpu_launches"],
+        "clocks": main_r["clocks"],
+        "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in main_r["kern"].items()},
+        other: {"value": o["value"], "ms_per_step": round(o["ms_per_step"], 5), "roofline": o["roofline"],
+                "path_roofline": o["path_roofline"], "e2e": o.get("e2e"), "gpu_launches": o["gpu_launches"],
+                "clocks": o["clocks"],
+                "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in o["kern"].items()}},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

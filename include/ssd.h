@@ -1,0 +1,187 @@
+/*
+ * ssd.h — C ABI of the B200 (sm_100a) Mamba-2 SSD chunked-scan library (libssd.so).
+ *
+ * The operation is the State Space Duality (SSD) scan of Mamba-2, computed by the
+ * five sub-modules named in "SSDi8: Accurate and Efficient 8-bit Quantization for
+ * State Space Duality" (ICLR 2026 paper notes, section "overall framework"):
+ * ChunkCumsum, ChunkState, StatePassing, ChunkBMM and ChunkScan (1 and 2).  It
+ * produces the result of the recurrence, per batch row b and head h,
+ *
+ *     h_t = exp(dt_t * A_h) * h_{t-1} + dt_t * x_t B_{g(h),t}^T      (h_t is P x N)
+ *     y_t = h_t C_{g(h),t} + D_h * x_t                                  (h_{-1} = 0)
+ *
+ * with g(h) = h / (H / G): B and C are stored per group and broadcast to blocks of
+ * H/G consecutive heads.
+ *
+ * Two precision paths:
+ *  - bf16 : bf16 inputs, fp32 accumulation, bf16 y, fp32 final state.
+ *  - W8A8 : the persistent-INT8 scheme of the same notes: B and C quantised once per
+ *           group (key design 3); ChunkState rebuilt as Q(LUT_state ⊙ X) x Q(B) with
+ *           INT32 accumulation (key design 1, eq. 4 and the reconstruction); the
+ *           state requantised to INT8 in registers with per-(H,P) scales, N left
+ *           unquantised, and passed between chunks with a fixed-point decay and a
+ *           shift by k = 7 (key design 2, eq. 6); ChunkBMM and ChunkScan1 on the
+ *           INT8 B, C and state; ChunkScan2 in floating point with the CB
+ *           dequantisation folded into LUT_Scan2.
+ *
+ * Conventions (all entry points):
+ *  - Tensors are dense, row-major, in the layouts given per argument; every device
+ *    pointer must be 16-byte aligned.  bf16 tensors are passed as uint16_t bit
+ *    patterns.  The caller owns every buffer; the library allocates no memory.
+ *  - Work is enqueued on `stream` and the call returns without synchronising.
+ *    Argument and shape errors are detected on the host before anything is
+ *    enqueued and are returned synchronously.  A failed launch returns SSD_ERR_CUDA.
+ *  - Supported shapes: chunk in {64, 128, 256}; (headdim P, dstate N) in
+ *    {(16,16), (64,128)}; nheads % ngroups == 0; any seqlen >= 0 (a final partial
+ *    chunk behaves as if padded with dt = 0, x = B = C = 0 tokens).  Other shapes
+ *    return SSD_ERR_UNSUPPORTED.
+ *  - Preconditions not checked (the values are not scanned): dt >= 0 and finite,
+ *    A <= 0, scales > 0 and finite.
+ *  - The initial state is zero.
+ *  - No C++ exception crosses this interface.
+ */
+#ifndef SSD_B200_H
+#define SSD_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, negative size, bad parameter */
+    SSD_ERR_UNSUPPORTED = 2,   /* shape outside the supported set */
+    SSD_ERR_WORKSPACE = 3,     /* workspace missing or smaller than ssd_workspace_bytes() */
+    SSD_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+    SSD_ERR_TIMEOUT = 5        /* a device-side bounded wait expired (read via ssd_workspace_status) */
+} ssd_status;
+
+typedef struct {
+    int batch;     /* B  >= 0 */
+    int seqlen;    /* L  >= 0 */
+    int nheads;    /* H  >= 1 */
+    int headdim;   /* P */
+    int ngroups;   /* G  >= 1, divides H */
+    int dstate;    /* N */
+    int chunk;     /* Q, the chunk length l of the notes */
+} ssd_shape;
+
+/* Static symmetric INT8 scales (step sizes: real value = code * scale), device fp32.
+ * Per-G for B and C, per-(H,P) for X_scaled and the state ("SSDi8" notes, key
+ * designs 2 and 3). */
+typedef struct {
+    const float* s_B;      /* [G] */
+    const float* s_C;      /* [G] */
+    const float* s_x;      /* [H*P], scale of X_scaled = LUT_state ⊙ x */
+    const float* s_s;      /* [H*P], scale of the INT8 state */
+    int decay_shift;       /* k of eq. 6 (S = 2^k); 1..14, the notes use 7 */
+} ssd_i8_params;
+
+/* Human-readable name of a status code (static string). */
+const char* ssd_status_string(ssd_status s);
+
+/* Bytes of device workspace that ssd_scan_fwd_bf16 (is_i8 = 0) or ssd_scan_fwd_i8
+ * (is_i8 = 1) need for `shape`; 0 for an invalid or unsupported shape.  The
+ * workspace holds the per-chunk cumulative decays, chunk states and passed states
+ * plus a device status word; its contents are private to the library. */
+size_t ssd_workspace_bytes(const ssd_shape* shape, int is_i8);
+
+/* ChunkBMM/ChunkScan inputs quantised once along G ("SSDi8" notes, key design 3):
+ *   Bq = clamp(rint(B * (1/s_B[g])), -127, 127), the same for C with s_C, in fp32 with
+ *   round-to-nearest-even; 1/s is an IEEE division.
+ * B, C : device bf16 [batch, seqlen, G, N].   s_B, s_C : device fp32 [G].
+ * Bq, Cq : device int8 [batch, seqlen, G, N], written. */
+ssd_status ssd_quantize_inputs(const ssd_shape* shape, const uint16_t* B, const uint16_t* C,
+                               const float* s_B, const float* s_C,
+                               int8_t* Bq, int8_t* Cq, cudaStream_t stream);
+
+/* bf16 SSD forward.
+ * x  : device bf16 [B, L, H, P]       dt : device fp32 [B, L, H] (after softplus, >= 0)
+ * A  : device fp32 [H] (<= 0)         B, C : device bf16 [B, L, G, N]
+ * D  : device fp32 [H]
+ * y  : device bf16 [B, L, H, P], written
+ * final_state : device fp32 [B, H, P, N], written (state after the last token)
+ * workspace : device, at least ssd_workspace_bytes(shape, 0) bytes. */
+ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const float* dt,
+                             const float* A, const uint16_t* B, const uint16_t* C,
+                             const float* D, uint16_t* y, float* final_state,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* W8A8 SSD forward on the INT8 inputs of ssd_quantize_inputs.
+ * x, dt, A, D, y : as in ssd_scan_fwd_bf16.   Bq, Cq : device int8 [B, L, G, N].
+ * params : host pointer to the scales (device arrays) and the decay shift k.
+ * final_state : device int8 [B, H, P, N], written; real value = code * s_s[h*P+p].
+ * workspace : device, at least ssd_workspace_bytes(shape, 1) bytes.
+ * Integer results (INT32 accumulators, INT8 states) are bit-exact with the
+ * library's specification; see ssd_debug_i8. */
+ssd_status ssd_scan_fwd_i8(const ssd_shape* shape, const uint16_t* x, const float* dt,
+                           const float* A, const int8_t* Bq, const int8_t* Cq, const float* D,
+                           const ssd_i8_params* params, uint16_t* y, int8_t* final_state,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Optional device buffers that ssd_scan_fwd_i8_debug fills with the W8A8
+ * intermediates (any may be NULL).  nc = ceil(L / Q); Lp = nc * Q.
+ *   Acs       fp32  [B, H, nc, Q]     inclusive cumulative dt*A per chunk
+ *   dq        int32 [B, H, nc]        decay codes rint(exp(Acs[Q-1]) * 2^k)
+ *   Xq        int8  [B, Lp, H, P]     quantised X_scaled
+ *   acc_state int32 [B, nc, H, P, N]  ChunkState accumulator Q(X_scaled)^T Q(B)
+ *   S8        int8  [B, nc, H, P, N]  requantised chunk states
+ *   H8        int8  [B, nc, H, P, N]  INT8 state entering each chunk
+ *   cb        int32 [B, nc, G, Q, Q]  ChunkBMM accumulator Cq Bq^T (entries with i <= j)
+ *   acc_scan1 int32 [B, Lp, H, P]     ChunkScan1 accumulator Cq H8^T */
+typedef struct {
+    float* Acs;
+    int32_t* dq;
+    int8_t* Xq;
+    int32_t* acc_state;
+    int8_t* S8;
+    int8_t* H8;
+    int32_t* cb;
+    int32_t* acc_scan1;
+} ssd_i8_debug;
+
+/* ssd_scan_fwd_i8 that also writes the intermediates named in `dbg` (host pointer). */
+ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, const float* dt,
+                                 const float* A, const int8_t* Bq, const int8_t* Cq,
+                                 const float* D, const ssd_i8_params* params, uint16_t* y,
+                                 int8_t* final_state, void* workspace, size_t workspace_bytes,
+                                 const ssd_i8_debug* dbg, cudaStream_t stream);
+
+/* Static calibration of the W8A8 scales over the first min(prefix, L) tokens of
+ * every batch row (symmetric, step size = amax / 127, amax = 0 gives 1):
+ *   s_B[g], s_C[g] : amax of |B|, |C| in group g
+ *   s_x[h*P+p]     : amax of |X_scaled| = |dt_j exp(Acs_{Q-1} - Acs_j) x_j|
+ *   s_s[h*P+p]     : amax over n of the chunk states S_c and the passed states
+ *                    H_1..H_nc of the prefix (fp32 bf16-path arithmetic)
+ * Inputs as in ssd_scan_fwd_bf16; outputs device fp32, written.  workspace: at
+ * least ssd_calibrate_workspace_bytes(shape, prefix) bytes. */
+size_t ssd_calibrate_workspace_bytes(const ssd_shape* shape, int prefix);
+ssd_status ssd_calibrate_i8(const ssd_shape* shape, int prefix, const uint16_t* x,
+                            const float* dt, const float* A, const uint16_t* B,
+                            const uint16_t* C, float* s_B, float* s_C, float* s_x, float* s_s,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Device status word of a workspace used by a previous call: synchronises `stream`,
+ * then returns SSD_OK or the error a kernel recorded (e.g. SSD_ERR_TIMEOUT), and
+ * clears it. */
+ssd_status ssd_workspace_status(void* workspace, cudaStream_t stream);
+
+/* Per-kernel timing (instrumentation, off by default).  While enabled, each kernel
+ * the entry points enqueue is bracketed by two CUDA events on the caller's stream.
+ * ssd_profile_read synchronises the recorded events and reports, for up to
+ * `capacity` kernel names, the accumulated milliseconds and the number of launches
+ * since the last reset; `count` receives the number of names known.  The name
+ * strings are owned by the library and stay valid until it is unloaded. */
+ssd_status ssd_profile_enable(int enable);
+ssd_status ssd_profile_read(int capacity, const char** names, double* ms, long long* calls, int* count);
+ssd_status ssd_profile_reset(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_B200_H */

@@ -1,0 +1,74 @@
+// common.cuh — shared device helpers of the SSD scan kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace ssd {
+
+// Problem dimensions as the kernels see them.  `Ls` is the row stride of the
+// token axis in elements of B*L-indexed tensors (equal to L except for the
+// calibration prefix, which runs on the first L tokens of rows of length Ls).
+struct Dims {
+    int B, L, H, P, G, N, Q, nc, hpg;
+    long long Ls;
+    __host__ __device__ long long Lp() const { return (long long)nc * Q; }
+};
+
+// Device status word values (first int32 of the workspace).
+enum : int { kStatusOk = 0, kStatusTimeout = 5 };
+
+// ---------------------------------------------------------------- bf16 helpers
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t v) {
+    return __uint_as_float(((uint32_t)v) << 16);
+}
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// ---------------------------------------------------------------- specified fp32 exp
+// exp(x) with a fixed sequence of individually rounded fp32 operations, so that the
+// W8A8 path's integer codes (X_scaled quantisation, decay codes) are reproducible
+// on any IEEE-754 machine.  Method: Cody-Waite range reduction x = k ln2 + r with
+// ln2 split into an 11-bit high part (k*ln2_hi exact for |k| < 2^13) and the rest,
+// then the degree-7 Taylor polynomial of exp(r) by Horner's rule, then scaling by
+// 2^k.  x < -87 gives 0; x is clamped to at most 88; exp(0) = 1 exactly.
+// No contraction into FMA: every step is an explicit _rn intrinsic.
+__device__ __forceinline__ float ssd_expf(float x) {
+    if (x < -87.0f) return 0.0f;
+    x = fminf(x, 88.0f);
+    const float kLog2e = 1.4426950408889634f;
+    const float kLn2Hi = 1420.0f / 2048.0f;
+    const float kLn2Lo = (float)(0.6931471805599453 - 1420.0 / 2048.0);
+    const float k = rintf(__fmul_rn(x, kLog2e));
+    const float r = __fsub_rn(__fsub_rn(x, __fmul_rn(k, kLn2Hi)), __fmul_rn(k, kLn2Lo));
+    float p = (float)(1.0 / 5040.0);
+    p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 720.0));
+    p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 120.0));
+    p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 24.0));
+    p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 6.0));
+    p = __fadd_rn(__fmul_rn(p, r), 0.5f);
+    p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+    p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+    int ki = (int)k;
+    ki = ki < -126 ? -126 : (ki > 127 ? 127 : ki);
+    const float two_k = __int_as_float((ki + 127) << 23);
+    return __fmul_rn(p, two_k);
+}
+
+// Symmetric INT8 code: clamp(rint(v * inv_scale), -127, 127), fp32 round-to-nearest-even.
+__device__ __forceinline__ int quant_i8(float v, float inv_scale) {
+    float q = rintf(__fmul_rn(v, inv_scale));
+    q = fminf(fmaxf(q, -127.0f), 127.0f);
+    return (int)q;
+}
+
+__device__ __forceinline__ int sat127(int v) { return v < -127 ? -127 : (v > 127 ? 127 : v); }
+
+// atomicMax on non-negative floats through their (monotone) bit patterns.
+__device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
+    atomicMax(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));
+}
+
+}  // namespace ssd

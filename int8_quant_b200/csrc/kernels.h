@@ -1,0 +1,84 @@
+// kernels.h — launchers of the SSD scan kernels (internal to libssd.so).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace ssd {
+
+// Workspace layout of one scan call (offsets in bytes, 256-byte aligned regions).
+struct WsLayout {
+    size_t status, acs, decay, states, passed, total;
+};
+WsLayout ws_layout(const Dims& d, bool i8);
+
+// Optional W8A8 intermediates (device pointers, any may be null).
+struct I8Debug {
+    float* Acs;
+    int32_t* dq;
+    int8_t* Xq;
+    int32_t* acc_state;
+    int8_t* S8;
+    int8_t* H8;
+    int32_t* cb;
+    int32_t* acc_scan1;
+};
+
+struct I8Scales {
+    const float* s_B;
+    const float* s_C;
+    const float* s_x;
+    const float* s_s;
+    int shift;
+};
+
+// a0: per-group INT8 quantisation of B and C.
+cudaError_t launch_quantize_bc(const Dims& d, const uint16_t* B, const uint16_t* C,
+                               const float* s_B, const float* s_C, int8_t* Bq, int8_t* Cq,
+                               cudaStream_t st);
+
+// a1: ChunkCumsum.  Writes Acs [B,H,nc,Q]; the bf16 path also the chunk decay
+// exp(Acs[Q-1]) (fp32 [B,H,nc]); the W8A8 path the decay codes (int32 [B,H,nc]).
+// Clears the workspace status word `status` (may be null) for the call.
+cudaError_t launch_cumsum(const Dims& d, const float* dt, const float* A, float* Acs,
+                          float* decay, int32_t* dq, int shift, int* status, cudaStream_t st);
+
+// a2: ChunkState.  bf16: fp32 states [B,nc,H,P,N]; W8A8: INT8 states.
+// amax_xs / amax_s (calibration only): per-(h,p) running max of |X_scaled| and |S_c|.
+cudaError_t launch_chunk_state_bf16(const Dims& d, const uint16_t* x, const float* dt,
+                                    const float* Acs, const uint16_t* B, float* S,
+                                    float* amax_xs, float* amax_s, cudaStream_t st);
+cudaError_t launch_chunk_state_i8(const Dims& d, const uint16_t* x, const float* dt,
+                                  const float* Acs, const int8_t* Bq, const I8Scales& sc,
+                                  int8_t* S8, const I8Debug* dbg, cudaStream_t st);
+
+// a3: StatePassing, sequential over chunks.
+//   bf16: H_{c+1} = decay_c * H_c + S_c in fp32; writes the state entering each
+//         chunk as bf16 (Hc) and/or fp32 (Hc32), the final state as fp32.
+//   W8A8: H_{c+1} = sat127(S8_c + ((dq_c * H_c + 2^(k-1)) >> k)).
+cudaError_t launch_state_passing_bf16(const Dims& d, const float* S, const float* decay,
+                                      uint16_t* Hc, float* final_state, float* amax_h,
+                                      cudaStream_t st);
+cudaError_t launch_state_passing_i8(const Dims& d, const int8_t* S8, const int32_t* dq, int shift,
+                                    int8_t* H8, int8_t* final_state, cudaStream_t st);
+
+// a4-a7: ChunkBMM + ChunkScan2 (diagonal) + ChunkScan1 (off-diagonal) + D skip.
+cudaError_t launch_chunk_scan_bf16(const Dims& d, const uint16_t* x, const float* dt,
+                                   const float* Acs, const uint16_t* B, const uint16_t* C,
+                                   const float* D, const uint16_t* Hc, uint16_t* y,
+                                   cudaStream_t st);
+cudaError_t launch_chunk_scan_i8(const Dims& d, const uint16_t* x, const float* dt,
+                                 const float* Acs, const int8_t* Bq, const int8_t* Cq,
+                                 const float* D, const I8Scales& sc, const int8_t* H8,
+                                 uint16_t* y, const I8Debug* dbg, cudaStream_t st);
+
+// Calibration helpers.
+cudaError_t launch_amax_bc(const Dims& d, const uint16_t* B, const uint16_t* C, float* amax_B,
+                           float* amax_C, cudaStream_t st);
+cudaError_t launch_amax_to_scale(float* v, int n, cudaStream_t st);
+cudaError_t launch_amax_pair_to_scale(const float* a1, const float* a2, float* out, int n,
+                                      cudaStream_t st);
+
+}  // namespace ssd

@@ -1,0 +1,122 @@
+// quantize.cu — a0 (per-group INT8 quantisation of B and C) and the calibration
+// reductions.  HBM-bound elementwise work: 16-byte loads of 8 bf16 values, 8-byte
+// stores of 8 int8 codes, grid sized to a multiple of the SM count.
+#include "kernels.h"
+
+namespace ssd {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__global__ void __launch_bounds__(kThreads)
+quantize_bc_kernel(const uint4* __restrict__ B, const uint4* __restrict__ C,
+                   const float* __restrict__ s_B, const float* __restrict__ s_C,
+                   uint2* __restrict__ Bq, uint2* __restrict__ Cq, long long nvec, int G, int N) {
+    const uint4* src = blockIdx.y == 0 ? B : C;
+    uint2* dst = blockIdx.y == 0 ? Bq : Cq;
+    const float* s = blockIdx.y == 0 ? s_B : s_C;
+    const int vec_per_group = N / 8;
+    for (long long i = blockIdx.x * (long long)kThreads + threadIdx.x; i < nvec;
+         i += (long long)gridDim.x * kThreads) {
+        const int g = (int)((i / vec_per_group) % G);
+        const float inv = __frcp_rn(__ldg(s + g));     // IEEE 1/s
+        const uint4 v = __ldg(src + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t out[2] = {0u, 0u};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint16_t bits = (uint16_t)(w[k >> 1] >> ((k & 1) * 16));
+            const int q = quant_i8(bf16_bits_to_float(bits), inv);
+            out[k >> 2] |= ((uint32_t)(q & 0xff)) << ((k & 3) * 8);
+        }
+        dst[i] = make_uint2(out[0], out[1]);
+    }
+}
+
+// Running amax of |B| and |C| per group over the first L tokens of each row.
+__global__ void __launch_bounds__(kThreads)
+amax_bc_kernel(const uint16_t* __restrict__ B, const uint16_t* __restrict__ C, float* amax_B,
+               float* amax_C, Dims d) {
+    const uint16_t* src = blockIdx.y == 0 ? B : C;
+    float* out = blockIdx.y == 0 ? amax_B : amax_C;
+    const long long per_row = (long long)d.L * d.G * d.N;
+    const long long total = per_row * d.B;
+    __shared__ float red[64];
+    for (int g = threadIdx.x; g < 64; g += kThreads) red[g] = 0.f;
+    __syncthreads();
+    for (long long i = blockIdx.x * (long long)kThreads + threadIdx.x; i < total;
+         i += (long long)gridDim.x * kThreads) {
+        const long long b = i / per_row, r = i % per_row;
+        const int g = (int)((r / d.N) % d.G);
+        const float v = fabsf(bf16_bits_to_float(src[b * d.Ls * d.G * d.N + r]));
+        atomic_max_nonneg(g < 64 ? &red[g] : out + g, v);
+    }
+    __syncthreads();
+    for (int g = threadIdx.x; g < d.G && g < 64; g += kThreads) atomic_max_nonneg(out + g, red[g]);
+}
+
+__global__ void amax_to_scale_kernel(float* v, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) {
+        const float a = v[i];
+        v[i] = a > 0.f ? __fdiv_rn(a, 127.0f) : 1.0f;
+    }
+}
+
+__global__ void amax_pair_to_scale_kernel(const float* a1, const float* a2, float* out, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) {
+        const float a = fmaxf(a1[i], a2[i]);
+        out[i] = a > 0.f ? __fdiv_rn(a, 127.0f) : 1.0f;
+    }
+}
+
+int grid_for(long long work, int per_block) {
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    long long blocks = (work + per_block - 1) / per_block;
+    long long cap = (long long)sms * 8;
+    if (blocks > cap) blocks = cap;
+    return (int)(blocks < 1 ? 1 : blocks);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_bc(const Dims& d, const uint16_t* B, const uint16_t* C,
+                               const float* s_B, const float* s_C, int8_t* Bq, int8_t* Cq,
+                               cudaStream_t st) {
+    const long long nvec = (long long)d.B * d.L * d.G * d.N / 8;
+    if (nvec == 0) return cudaSuccess;
+    dim3 grid(grid_for(nvec, kThreads), 2);
+    quantize_bc_kernel<<<grid, kThreads, 0, st>>>(reinterpret_cast<const uint4*>(B),
+                                                  reinterpret_cast<const uint4*>(C), s_B, s_C,
+                                                  reinterpret_cast<uint2*>(Bq),
+                                                  reinterpret_cast<uint2*>(Cq), nvec, d.G, d.N);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_amax_bc(const Dims& d, const uint16_t* B, const uint16_t* C, float* amax_B,
+                           float* amax_C, cudaStream_t st) {
+    const long long total = (long long)d.B * d.L * d.G * d.N;
+    if (total == 0) return cudaSuccess;
+    dim3 grid(grid_for(total, kThreads), 2);
+    amax_bc_kernel<<<grid, kThreads, 0, st>>>(B, C, amax_B, amax_C, d);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_amax_to_scale(float* v, int n, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    amax_to_scale_kernel<<<(n + 255) / 256, 256, 0, st>>>(v, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_amax_pair_to_scale(const float* a1, const float* a2, float* out, int n,
+                                      cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    amax_pair_to_scale_kernel<<<(n + 255) / 256, 256, 0, st>>>(a1, a2, out, n);
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

@@ -1,0 +1,101 @@
+"""The C-ABI library loads and exports what include/ssd.h declares; host-side validation (no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import int8_quant_b200 as iq
+from int8_quant_b200 import ssd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "ssd.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssd_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_header_declares_the_binding_names():
+    assert sorted(ssd.EXPORTS) == _declared()
+
+
+def test_library_exports_every_declared_symbol():
+    lib = iq.library()
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings():
+    lib = iq.library()
+    for code, name in ssd.STATUS_NAMES.items():
+        assert lib.ssd_status_string(code).decode().startswith(name)
+
+
+@pytest.mark.parametrize("shape,ok", [
+    ((8, 8192, 80, 64, 1, 128, 256), True),
+    ((1, 256, 4, 16, 1, 16, 64), True),
+    ((1, 100, 4, 64, 2, 128, 128), True),
+    ((0, 0, 4, 64, 1, 128, 256), True),
+    ((1, 256, 4, 32, 1, 16, 64), False),     # unsupported (P, N)
+    ((1, 256, 4, 64, 1, 128, 96), False),    # unsupported chunk
+    ((1, 256, 6, 64, 4, 128, 256), False),   # H % G != 0
+    ((-1, 256, 4, 64, 1, 128, 256), False),
+])
+def test_workspace_bytes_validates_shapes(shape, ok):
+    s = iq.SsdShape.of(*shape)
+    assert (iq.ssd_workspace_bytes(s, False) > 0) == ok
+    assert (iq.ssd_workspace_bytes(s, True) > 0) == ok
+
+
+def test_workspace_grows_with_the_problem_and_i8_is_smaller():
+    a = iq.ssd_workspace_bytes(iq.SsdShape.of(1, 1024, 8, 64, 1, 128, 256), False)
+    b = iq.ssd_workspace_bytes(iq.SsdShape.of(2, 1024, 8, 64, 1, 128, 256), False)
+    c = iq.ssd_workspace_bytes(iq.SsdShape.of(2, 1024, 8, 64, 1, 128, 256), True)
+    assert b > a and c < b
+
+
+def _fake(n=0x10000):
+    return ctypes.c_void_p(n)        # aligned, never dereferenced: every call below fails validation
+
+
+def test_invalid_arguments_fail_before_any_launch():
+    lib = iq.library()
+    s = iq.SsdShape.of(1, 256, 4, 64, 1, 128, 256)
+    f = _fake()
+    ws = iq.ssd_workspace_bytes(s, False)
+    # null x
+    st = lib.ssd_scan_fwd_bf16(ctypes.byref(s), None, f, f, f, f, f, f, f, f, ws, None)
+    assert st == 1
+    # misaligned y
+    st = lib.ssd_scan_fwd_bf16(ctypes.byref(s), f, f, f, f, f, f, _fake(0x10002), f, f, ws, None)
+    assert st == 1
+    # workspace too small / missing
+    assert lib.ssd_scan_fwd_bf16(ctypes.byref(s), f, f, f, f, f, f, f, f, f, ws - 1, None) == 3
+    assert lib.ssd_scan_fwd_bf16(ctypes.byref(s), f, f, f, f, f, f, f, f, None, ws, None) == 3
+    # unsupported shape
+    s2 = iq.SsdShape.of(1, 256, 4, 32, 1, 16, 64)
+    assert lib.ssd_scan_fwd_bf16(ctypes.byref(s2), f, f, f, f, f, f, f, f, f, 1 << 30, None) == 2
+    # W8A8: missing params, bad shift
+    wsi = iq.ssd_workspace_bytes(s, True)
+    assert lib.ssd_scan_fwd_i8(ctypes.byref(s), f, f, f, f, f, f, None, f, f, f, wsi, None) == 1
+    p = iq.SsdI8Params(0x10000, 0x10000, 0x10000, 0x10000, 0)
+    assert lib.ssd_scan_fwd_i8(ctypes.byref(s), f, f, f, f, f, f, ctypes.byref(p), f, f, f, wsi, None) == 1
+    p.decay_shift = 15
+    assert lib.ssd_scan_fwd_i8(ctypes.byref(s), f, f, f, f, f, f, ctypes.byref(p), f, f, f, wsi, None) == 1
+    # quantize: null outputs
+    assert lib.ssd_quantize_inputs(ctypes.byref(s), f, f, f, f, None, f, None) == 1
+    # calibration: workspace too small
+    cw = iq.ssd_calibrate_workspace_bytes(s, 512)
+    assert cw > 0
+    assert lib.ssd_calibrate_i8(ctypes.byref(s), 512, f, f, f, f, f, f, f, f, f, f, cw - 1, None) == 3
+    assert lib.ssd_calibrate_i8(ctypes.byref(s), -1, f, f, f, f, f, f, f, f, f, f, cw, None) == 1
+
+
+def test_null_shape_is_rejected():
+    lib = iq.library()
+    assert lib.ssd_workspace_bytes(None, 0) == 0
+    f = _fake()
+    assert lib.ssd_scan_fwd_bf16(None, f, f, f, f, f, f, f, f, f, 1 << 20, None) == 1
