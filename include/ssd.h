@@ -111,13 +111,38 @@ ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const fl
                              const float* D, uint16_t* y, float* final_state,
                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Size of the library's fixed device scratch used by ssd_scan_fwd_bf16_static. */
+#define SSD_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* The bf16 SSD forward without a caller-provided workspace, for callers that cannot
+ * allocate device memory (an allocator or arena that owns all device memory, a
+ * plugin or embedded runtime that may not call cudaMalloc, a latency-critical thread
+ * that must not take allocation locks).  The paper notes have no counterpart: this
+ * is a packaging variant of ssd_scan_fwd_bf16, with the same arguments minus the
+ * workspace and the same results.
+ *  - Scratch lives in a fixed SSD_STATIC_SCRATCH_BYTES (32 MiB) array in the
+ *    library's device memory, held by every GPU that loads the library until the
+ *    process exits.  A shape whose ssd_workspace_bytes(shape, 0) exceeds it is
+ *    rejected with SSD_ERR_WORKSPACE before anything is enqueued.
+ *  - Nothing is allocated: no cudaMalloc/cudaFree or allocating library routine.
+ *  - The first call on each device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any stream
+ *    capture.
+ *  - All calls share the one array, which keeps the last call's contents (each call
+ *    rewrites what it reads).  Calls whose GPU work overlaps (other streams, other
+ *    host threads) race on it: serialise them. */
+ssd_status ssd_scan_fwd_bf16_static(const ssd_shape* shape, const uint16_t* x, const float* dt,
+                                    const float* A, const uint16_t* B, const uint16_t* C,
+                                    const float* D, uint16_t* y, float* final_state,
+                                    cudaStream_t stream);
+
 /* W8A8 SSD forward on the INT8 inputs of ssd_quantize_inputs.
  * x, dt, A, D, y : as in ssd_scan_fwd_bf16.   Bq, Cq : device int8 [B, L, G, N].
  * params : host pointer to the scales (device arrays) and the decay shift k.
  * final_state : device int8 [B, H, P, N], written; real value = code * s_s[h*P+p].
  * workspace : device, at least ssd_workspace_bytes(shape, 1) bytes.
  * Integer results (INT32 accumulators, INT8 states) are bit-exact with the
- * library's specification; see ssd_debug_i8. */
+ * library's specification; see ssd_scan_fwd_i8_debug. */
 ssd_status ssd_scan_fwd_i8(const ssd_shape* shape, const uint16_t* x, const float* dt,
                            const float* A, const int8_t* Bq, const int8_t* Cq, const float* D,
                            const ssd_i8_params* params, uint16_t* y, int8_t* final_state,

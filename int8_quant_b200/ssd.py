@@ -21,7 +21,10 @@ STATUS_NAMES = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
 EXPORTS = ("ssd_status_string", "ssd_workspace_bytes", "ssd_quantize_inputs", "ssd_scan_fwd_bf16",
            "ssd_scan_fwd_i8", "ssd_scan_fwd_i8_debug", "ssd_calibrate_workspace_bytes",
            "ssd_calibrate_i8", "ssd_workspace_status", "ssd_profile_enable", "ssd_profile_read",
-           "ssd_profile_reset")
+           "ssd_profile_reset", "ssd_scan_fwd_bf16_static")
+
+# Size of the library's fixed device scratch used by ssd_scan_fwd_bf16_static.
+STATIC_SCRATCH_BYTES = 32 << 20
 
 
 class SsdShape(ctypes.Structure):
@@ -73,6 +76,8 @@ def _lib():
         lib.ssd_quantize_inputs.argtypes = [sp, P, P, P, P, P, P, P]
         lib.ssd_scan_fwd_bf16.restype = I
         lib.ssd_scan_fwd_bf16.argtypes = [sp, P, P, P, P, P, P, P, P, P, S, P]
+        lib.ssd_scan_fwd_bf16_static.restype = I
+        lib.ssd_scan_fwd_bf16_static.argtypes = [sp, P, P, P, P, P, P, P, P, P]
         lib.ssd_scan_fwd_i8.restype = I
         lib.ssd_scan_fwd_i8.argtypes = [sp, P, P, P, P, P, P, ctypes.POINTER(SsdI8Params), P, P, P, S, P]
         lib.ssd_scan_fwd_i8_debug.restype = I
@@ -140,6 +145,15 @@ def ssd_scan_fwd_bf16(shape, x, dt, A, B, C, D, y, final_state, workspace, strea
     _check("ssd_scan_fwd_bf16", _lib().ssd_scan_fwd_bf16(
         ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
         _ptr(final_state), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def ssd_scan_fwd_bf16_static(shape, x, dt, A, B, C, D, y, final_state, stream=None):
+    """ssd_scan_fwd_bf16 without a workspace argument: the library's fixed 32 MiB device
+    scratch is used instead, for callers that cannot allocate device memory.  Calls
+    share that scratch, so calls whose GPU work overlaps must be serialised."""
+    _check("ssd_scan_fwd_bf16_static", _lib().ssd_scan_fwd_bf16_static(
+        ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y), _ptr(final_state),
+        _stream(stream)))
 
 
 def i8_params(s_B, s_C, s_x, s_s, decay_shift=7) -> SsdI8Params:
