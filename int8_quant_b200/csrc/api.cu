@@ -39,6 +39,10 @@ ssd_status make_dims(const ssd_shape* s, Dims* d) {
     return SSD_OK;
 }
 
+// Shapes served by the tensor-core kernels; the (16,16) test shape uses the
+// CUDA-core kernels.
+bool tensor_core_shape(const Dims& d) { return d.P == 64 && d.N == 128; }
+
 ssd_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
 
 #define SSD_TRY(expr)                                  \
@@ -59,6 +63,8 @@ WsLayout ws_layout(const Dims& d, bool i8) {
     size_t off = 0;
     w.status = off;  off += 256;
     w.acs = off;     off += align256(chains * d.nc * d.Q * sizeof(float));
+    w.lut = off;     off += align256(chains * d.nc * d.Q * sizeof(float));   // LUT_state
+    w.dtc = off;     off += align256(chains * d.nc * d.Q * sizeof(float));   // dt, chunk-major
     w.decay = off;   off += align256(chains * d.nc * sizeof(float));   // fp32 decay or int32 code
     w.states = off;  off += align256(states * (i8 ? 1 : sizeof(float)));
     w.passed = off;  off += align256(states * (i8 ? 1 : sizeof(uint16_t)));
@@ -196,8 +202,14 @@ ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const fl
     float* decay = at<float>(workspace, w.decay);
     float* S = at<float>(workspace, w.states);
     uint16_t* Hc = at<uint16_t>(workspace, w.passed);
-    SSD_STAGE("chunk_cumsum", launch_cumsum(d, dt, A, Acs, decay, nullptr, 0, at<int>(workspace, w.status), stream));
-    SSD_STAGE("chunk_state", launch_chunk_state_bf16(d, x, dt, Acs, B, S, nullptr, nullptr, stream));
+    float* lut = at<float>(workspace, w.lut);
+    float* dtc = at<float>(workspace, w.dtc);
+    int* status = at<int>(workspace, w.status);
+    SSD_STAGE("chunk_cumsum", launch_cumsum(d, dt, A, Acs, decay, nullptr, 0, status, lut, dtc, stream));
+    if (tensor_core_shape(d))
+        SSD_STAGE("chunk_state", launch_chunk_state_tc(d, false, x, B, lut, I8Scales{}, S, nullptr, nullptr, status, stream));
+    else
+        SSD_STAGE("chunk_state", launch_chunk_state_bf16(d, x, dt, Acs, B, S, nullptr, nullptr, stream));
     SSD_STAGE("state_passing", launch_state_passing_bf16(d, S, decay, Hc, final_state, nullptr, stream));
     SSD_STAGE("chunk_scan", launch_chunk_scan_bf16(d, x, dt, Acs, B, C, D, Hc, y, stream));
     return SSD_OK;
@@ -229,8 +241,14 @@ ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, cons
     I8Scales sc{params->s_B, params->s_C, params->s_x, params->s_s, params->decay_shift};
     I8Debug dd{};
     if (dbg) dd = I8Debug{dbg->Acs, dbg->dq, dbg->Xq, dbg->acc_state, dbg->S8, dbg->H8, dbg->cb, dbg->acc_scan1};
-    SSD_STAGE("chunk_cumsum", launch_cumsum(d, dt, A, Acs, nullptr, dq, sc.shift, at<int>(workspace, w.status), stream));
-    SSD_STAGE("chunk_state", launch_chunk_state_i8(d, x, dt, Acs, Bq, sc, S8, dbg ? &dd : nullptr, stream));
+    float* lut = at<float>(workspace, w.lut);
+    float* dtc = at<float>(workspace, w.dtc);
+    int* status = at<int>(workspace, w.status);
+    SSD_STAGE("chunk_cumsum", launch_cumsum(d, dt, A, Acs, nullptr, dq, sc.shift, status, lut, dtc, stream));
+    if (tensor_core_shape(d))
+        SSD_STAGE("chunk_state", launch_chunk_state_tc(d, true, x, Bq, lut, sc, nullptr, S8, dbg ? &dd : nullptr, status, stream));
+    else
+        SSD_STAGE("chunk_state", launch_chunk_state_i8(d, x, dt, Acs, Bq, sc, S8, dbg ? &dd : nullptr, stream));
     SSD_STAGE("state_passing", launch_state_passing_i8(d, S8, dq, sc.shift, H8, final_state, stream));
     SSD_STAGE("chunk_scan", launch_chunk_scan_i8(d, x, dt, Acs, Bq, Cq, D, sc, H8, y, dbg ? &dd : nullptr, stream));
     if (dbg) {
@@ -303,7 +321,7 @@ ssd_status ssd_calibrate_i8(const ssd_shape* shape, int prefix, const uint16_t* 
         float* S = at<float>(workspace, w.states);
         float* fin = at<float>(workspace, fin_off);
         SSD_TRY(launch_amax_bc(p, B, C, aB, aC, stream));
-        SSD_TRY(launch_cumsum(p, dt, A, Acs, decay, nullptr, 0, nullptr, stream));
+        SSD_TRY(launch_cumsum(p, dt, A, Acs, decay, nullptr, 0, nullptr, nullptr, nullptr, stream));
         SSD_TRY(launch_chunk_state_bf16(p, x, dt, Acs, B, S, ax, as, stream));
         SSD_TRY(launch_state_passing_bf16(p, S, decay, nullptr, fin, ah, stream));
     }

@@ -1,6 +1,9 @@
 // cumsum.cu — a1, ChunkCumsum: Acs[b,h,c,j] = sum_{i<=j} dt[b,cQ+i,h] * A[h] within each
 // chunk, plus the chunk decay exp(Acs[Q-1]) (bf16 path) or its fixed-point code
-// rint(exp(Acs[Q-1]) * 2^k) (W8A8 path, eq. 6 of the SSDi8 notes).
+// rint(exp(Acs[Q-1]) * 2^k) (W8A8 path, eq. 6 of the SSDi8 notes).  Optionally also
+// LUT_state[b,h,c,j] = dt_j * exp(Acs[Q-1] - Acs[j]) (eq. 4; the W8A8 path uses the
+// specified fp32 exp so that X_scaled's codes are reproducible) and dt in the same
+// chunk-major layout, so that the tensor-core kernels read both contiguously.
 //
 // One CTA per (chunk, block of 32 heads, batch row).  dt rows of the chunk are
 // staged in shared memory with coalesced 128-byte row reads (32 heads x fp32),
@@ -22,7 +25,7 @@ template <bool kI8>
 __global__ void __launch_bounds__(kThreads)
 cumsum_kernel(Dims d, const float* __restrict__ dt, const float* __restrict__ A,
               float* __restrict__ Acs, float* __restrict__ decay, int32_t* __restrict__ dq,
-              int shift, int* __restrict__ status) {
+              int shift, int* __restrict__ status, float* __restrict__ lut, float* __restrict__ dtc) {
     // this call's kernels record device-side errors in the workspace status word
     if (status && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) *status = kStatusOk;
     extern __shared__ float tile[];                 // [Q][kHeadsPerCta + 1]
@@ -60,14 +63,29 @@ cumsum_kernel(Dims d, const float* __restrict__ dt, const float* __restrict__ A,
         }
         float e = __shfl_up_sync(0xffffffffu, v, 1);
         if (lane == 0) e = 0.f;
-        float* out = Acs + (((long long)b * d.H + h) * d.nc + c) * Q + lane * m;
+        const long long row = (((long long)b * d.H + h) * d.nc + c) * Q + lane * m;
+        float* out = Acs + row;
+        float acs[8];
         float last = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             if (i < m) {
                 const float r = __fadd_rn(e, s[i]);
                 out[i] = r;
+                acs[i] = r;
                 last = r;
+            }
+        }
+        last = __shfl_sync(0xffffffffu, last, 31);          // Acs[Q-1]
+        if (lut) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (i < m) {
+                    const float dtv = tile[(lane * m + i) * ld + k];
+                    lut[row + i] = kI8 ? __fmul_rn(dtv, ssd_expf(__fsub_rn(last, acs[i])))
+                                       : dtv * expf(last - acs[i]);
+                    if (dtc) dtc[row + i] = dtv;
+                }
             }
         }
         if (lane == 31) {
@@ -84,16 +102,17 @@ cumsum_kernel(Dims d, const float* __restrict__ dt, const float* __restrict__ A,
 }  // namespace
 
 cudaError_t launch_cumsum(const Dims& d, const float* dt, const float* A, float* Acs,
-                          float* decay, int32_t* dq, int shift, int* status, cudaStream_t st) {
+                          float* decay, int32_t* dq, int shift, int* status, float* lut, float* dtc,
+                          cudaStream_t st) {
     if (d.B == 0 || d.nc == 0) return cudaSuccess;
     dim3 grid(d.nc, (d.H + kHeadsPerCta - 1) / kHeadsPerCta, d.B);
     const size_t smem = (size_t)d.Q * (kHeadsPerCta + 1) * sizeof(float);
     if (dq) {
         cudaFuncSetAttribute(cumsum_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        cumsum_kernel<true><<<grid, kThreads, smem, st>>>(d, dt, A, Acs, decay, dq, shift, status);
+        cumsum_kernel<true><<<grid, kThreads, smem, st>>>(d, dt, A, Acs, decay, dq, shift, status, lut, dtc);
     } else {
         cudaFuncSetAttribute(cumsum_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        cumsum_kernel<false><<<grid, kThreads, smem, st>>>(d, dt, A, Acs, decay, dq, shift, status);
+        cumsum_kernel<false><<<grid, kThreads, smem, st>>>(d, dt, A, Acs, decay, dq, shift, status, lut, dtc);
     }
     return cudaGetLastError();
 }

@@ -1,6 +1,7 @@
 // kernels.h — launchers of the SSD scan kernels (internal to libssd.so).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -10,7 +11,7 @@ namespace ssd {
 
 // Workspace layout of one scan call (offsets in bytes, 256-byte aligned regions).
 struct WsLayout {
-    size_t status, acs, decay, states, passed, total;
+    size_t status, acs, lut, dtc, decay, states, passed, total;
 };
 WsLayout ws_layout(const Dims& d, bool i8);
 
@@ -41,9 +42,11 @@ cudaError_t launch_quantize_bc(const Dims& d, const uint16_t* B, const uint16_t*
 
 // a1: ChunkCumsum.  Writes Acs [B,H,nc,Q]; the bf16 path also the chunk decay
 // exp(Acs[Q-1]) (fp32 [B,H,nc]); the W8A8 path the decay codes (int32 [B,H,nc]).
-// Clears the workspace status word `status` (may be null) for the call.
+// Clears the workspace status word `status` (may be null) for the call.  `lut`
+// (LUT_state) and `dtc` (dt) are optional [B,H,nc,Q] outputs.
 cudaError_t launch_cumsum(const Dims& d, const float* dt, const float* A, float* Acs,
-                          float* decay, int32_t* dq, int shift, int* status, cudaStream_t st);
+                          float* decay, int32_t* dq, int shift, int* status, float* lut, float* dtc,
+                          cudaStream_t st);
 
 // a2: ChunkState.  bf16: fp32 states [B,nc,H,P,N]; W8A8: INT8 states.
 // amax_xs / amax_s (calibration only): per-(h,p) running max of |X_scaled| and |S_c|.
@@ -73,6 +76,19 @@ cudaError_t launch_chunk_scan_i8(const Dims& d, const uint16_t* x, const float* 
                                  const float* Acs, const int8_t* Bq, const int8_t* Cq,
                                  const float* D, const I8Scales& sc, const int8_t* H8,
                                  uint16_t* y, const I8Debug* dbg, cudaStream_t st);
+
+// 3D TMA tensor map over a [d2][d1][d0] tensor of bf16 (or int8 when is_i8) with the
+// given byte strides of dims 1 and 2, a box of box1 x box0 elements, and a swizzle.
+bool make_tmap_3d(CUtensorMap* m, bool is_i8, const void* base, unsigned long long d0, unsigned long long d1,
+                  unsigned long long d2, unsigned long long stride1_bytes, unsigned long long stride2_bytes,
+                  unsigned box0, unsigned box1, CUtensorMapSwizzle swizzle);
+
+// Tensor-core ChunkState for P = 64, N = 128: one CTA per (head, chunk, batch row)
+// computes the chunk state transposed, S^T[n,p] = sum_j B[j,n] X_scaled[j,p], with
+// tcgen05 (kind::f16, or kind::i8 on Xq and Bq).  `lut` is LUT_state [B,H,nc,Q].
+cudaError_t launch_chunk_state_tc(const Dims& d, bool i8, const uint16_t* x, const void* Bmat,
+                                  const float* lut, const I8Scales& sc, float* S, int8_t* S8,
+                                  const I8Debug* dbg, int* status, cudaStream_t st);
 
 // Calibration helpers.
 cudaError_t launch_amax_bc(const Dims& d, const uint16_t* B, const uint16_t* C, float* amax_B,
