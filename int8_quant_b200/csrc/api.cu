@@ -43,6 +43,9 @@ ssd_status make_dims(const ssd_shape* s, Dims* d) {
 // CUDA-core kernels.
 bool tensor_core_shape(const Dims& d) { return d.P == 64 && d.N == 128; }
 
+// Heads that share one ChunkBMM result in the tensor-core ChunkScan.
+constexpr int kHeadsPerScanCta = 8;
+
 ssd_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
 
 #define SSD_TRY(expr)                                  \
@@ -211,7 +214,11 @@ ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const fl
     else
         SSD_STAGE("chunk_state", launch_chunk_state_bf16(d, x, dt, Acs, B, S, nullptr, nullptr, stream));
     SSD_STAGE("state_passing", launch_state_passing_bf16(d, S, decay, Hc, final_state, nullptr, stream));
-    SSD_STAGE("chunk_scan", launch_chunk_scan_bf16(d, x, dt, Acs, B, C, D, Hc, y, stream));
+    if (tensor_core_shape(d))
+        SSD_STAGE("chunk_scan", launch_chunk_scan_tc(d, false, x, B, C, Acs, dtc, D, I8Scales{}, Hc, y, nullptr,
+                                                     kHeadsPerScanCta, status, stream));
+    else
+        SSD_STAGE("chunk_scan", launch_chunk_scan_bf16(d, x, dt, Acs, B, C, D, Hc, y, stream));
     return SSD_OK;
 }
 
@@ -250,7 +257,11 @@ ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, cons
     else
         SSD_STAGE("chunk_state", launch_chunk_state_i8(d, x, dt, Acs, Bq, sc, S8, dbg ? &dd : nullptr, stream));
     SSD_STAGE("state_passing", launch_state_passing_i8(d, S8, dq, sc.shift, H8, final_state, stream));
-    SSD_STAGE("chunk_scan", launch_chunk_scan_i8(d, x, dt, Acs, Bq, Cq, D, sc, H8, y, dbg ? &dd : nullptr, stream));
+    if (tensor_core_shape(d))
+        SSD_STAGE("chunk_scan", launch_chunk_scan_tc(d, true, x, Bq, Cq, Acs, dtc, D, sc, H8, y, dbg ? &dd : nullptr,
+                                                     kHeadsPerScanCta, status, stream));
+    else
+        SSD_STAGE("chunk_scan", launch_chunk_scan_i8(d, x, dt, Acs, Bq, Cq, D, sc, H8, y, dbg ? &dd : nullptr, stream));
     if (dbg) {
         const size_t chains = (size_t)d.B * d.H;
         const size_t states = (size_t)d.B * d.nc * d.H * d.P * d.N;

@@ -83,6 +83,18 @@ bool make_tmap_3d(CUtensorMap* m, bool is_i8, const void* base, unsigned long lo
                   unsigned long long d2, unsigned long long stride1_bytes, unsigned long long stride2_bytes,
                   unsigned box0, unsigned box1, CUtensorMapSwizzle swizzle);
 
+bool make_tmap_2d(CUtensorMap* m, bool is_i8, const void* base, unsigned long long d0, unsigned long long d1,
+                  unsigned long long stride1_bytes, unsigned box0, unsigned box1, CUtensorMapSwizzle swizzle);
+
+// Tensor-core ChunkBMM + ChunkScan2 + ChunkScan1 + D skip for P = 64, N = 128: one
+// CTA per (chunk, batch row, block of up to `heads_per_cta` heads of one group).
+// `Hc` is the state entering each chunk (bf16 or int8 [B,nc,H,P,N]); Acs and dtc
+// are [B,H,nc,Q].
+cudaError_t launch_chunk_scan_tc(const Dims& d, bool i8, const uint16_t* x, const void* Bmat,
+                                 const void* Cmat, const float* Acs, const float* dtc, const float* D,
+                                 const I8Scales& sc, const void* Hc, uint16_t* y, const I8Debug* dbg,
+                                 int heads_per_cta, int* status, cudaStream_t st);
+
 // Tensor-core ChunkState for P = 64, N = 128: one CTA per (head, chunk, batch row)
 // computes the chunk state transposed, S^T[n,p] = sum_j B[j,n] X_scaled[j,p], with
 // tcgen05 (kind::f16, or kind::i8 on Xq and Bq).  `lut` is LUT_state [B,H,nc,Q].

@@ -42,4 +42,18 @@ bool make_tmap_3d(CUtensorMap* m, bool is_i8, const void* base, unsigned long lo
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_2d(CUtensorMap* m, bool is_i8, const void* base, unsigned long long d0, unsigned long long d1,
+                  unsigned long long stride1_bytes, unsigned box0, unsigned box1, CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {d0, d1};
+    const cuuint64_t strides[1] = {stride1_bytes};
+    const cuuint32_t box[2] = {box0, box1};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, is_i8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace ssd
