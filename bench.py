@@ -313,7 +313,8 @@ def run_ours(args, rank, world, dist):
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4), "steps": n}
 
     results = {}
-    for path in (args.path, "bf16" if args.path == "w8a8" else "w8a8"):
+    paths = (args.path,) if args.only_path else (args.path, "bf16" if args.path == "w8a8" else "w8a8")
+    for path in paths:
         ms, kern, clocks = timed(path)
         launches = sum(c for _, c in kern.values())
         alg = path_bytes(w, path)
@@ -337,6 +338,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2-2.7b", choices=sorted(WORKLOADS))
     ap.add_argument("--path", choices=["w8a8", "bf16"], default="w8a8")
+    ap.add_argument("--only-path", action="store_true", help="time only --path (profiling runs)")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")
+    ap.add_argument("--seqlen", type=int, default=None, help="override the workload's length (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -346,6 +350,11 @@ def main():
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.batch is not None or args.seqlen is not None:
+        base = WORKLOADS[args.workload]
+        name = f"{base.name}-b{args.batch or base.batch}-l{args.seqlen or base.seqlen}"
+        WORKLOADS[name] = base.with_(name=name, batch=args.batch or base.batch, seqlen=args.seqlen or base.seqlen)
+        args.workload = name
     w = WORKLOADS[args.workload]
 
     if args.impl == "reference":
@@ -405,7 +414,7 @@ def main():
         return
     main_r = res[args.path]
     other = "bf16" if args.path == "w8a8" else "w8a8"
-    o = res[other]
+    o = res.get(other)
     line = {
         "metric": METRIC, "value": main_r["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(main_r["ms_per_step"], 5), "higher_is_better": True,
@@ -421,11 +430,12 @@ def main():
         "cpu_baseline": cpu, "e2e": main_r.get("e2e"), "gpu_launches": main_r["gpu_launches"],
         "clocks": main_r["clocks"],
         "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in main_r["kern"].items()},
-        other: {"value": o["value"], "ms_per_step": round(o["ms_per_step"], 5), "roofline": o["roofline"],
-                "path_roofline": o["path_roofline"], "e2e": o.get("e2e"), "gpu_launches": o["gpu_launches"],
-                "clocks": o["clocks"],
-                "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in o["kern"].items()}},
     }
+    if o is not None:
+        line[other] = {"value": o["value"], "ms_per_step": round(o["ms_per_step"], 5), "roofline": o["roofline"],
+                       "path_roofline": o["path_roofline"], "e2e": o.get("e2e"), "gpu_launches": o["gpu_launches"],
+                       "clocks": o["clocks"],
+                       "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in o["kern"].items()}}
     print(json.dumps(line), flush=True)
 
 
