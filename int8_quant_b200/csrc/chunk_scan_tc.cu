@@ -22,12 +22,16 @@
 //               the masked matrix as they arrive.
 //   warps 2-9   builders, two sets of four (one warp per TMEM lane quarter):
 //               M[j,i] = CB[j,i] exp(Acs_j - Acs_i) dt_i, 64 columns per piece, into
-//               a 4-slot ring of 128-byte-swizzled K-major tiles.  Below the 64-row
+//               a 2-slot ring in TMEM (bf16 pairs), which the y += M x MMAs read as
+//               their A operand: M never touches shared memory, whose bandwidth
+//               (128 B/clk) the skinny N = 64 MMAs already saturate.  Below the 64-row
 //               diagonal blocks the decay factorises through the block boundary r:
 //               exp(Acs_j - Acs_r) * exp(Acs_r - Acs_i), both <= 1, so only the
 //               diagonal blocks take an exponential per element.
 //   warps 10-13 scalers: ChunkScan1 rows times exp(Acs_j) in TMEM (W8A8: dequantise).
-//   warps 14-17 storers: y + D x, rounded to bf16 over the x tile, stored by TMA.
+//   warps 14-17 storers: y + D x, rounded to bf16 over the x tile, stored by TMA
+//               (a warp's rows are 10 KB apart in y, so stores from registers would
+//               not coalesce).
 // Every wait is bounded; an expired wait raises a shared abort flag that ends all
 // roles, records SSD_ERR_TIMEOUT in the status word, and the CTA frees TMEM.
 #include "kernels.h"
@@ -46,7 +50,7 @@ constexpr int kBuilderThreads = 256;
 constexpr int kScaleWarp0 = 10;
 constexpr int kStoreWarp0 = 14;
 constexpr int kEpiThreads = 128;
-constexpr int kRing = 4;
+constexpr int kRing = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 enum : uint32_t { kIdBuild = 1, kIdScale = 2, kIdStore = 3 };
 
@@ -56,22 +60,18 @@ struct Cfg {
     static constexpr int CROWS = Q >= 128 ? Q : 128;             // C rows loaded (Q = 64: ghost rows)
     static constexpr int NCB0 = Q >= 128 ? 128 : Q;              // CB columns of tile 0
     static constexpr int NPIECE = JT == 2 ? 6 : NCB0 / 64;       // 64-column pieces of M per head
-    // TMEM columns: fp32 CB at [128, ...), packed CB at [0, 192), y slots at 256 + 128 s
-    static constexpr uint32_t CBF = 128, CBP0 = 0, CBP1 = 64, YCOL = 256, TMEM_COLS = 512;
+    // TMEM columns: packed CB at [0, 192), M ring at [192, 256), y slots at 256 + 128 s;
+    // the fp32 CB accumulators use [128, ...) before they are packed
+    static constexpr uint32_t CBF = 128, CBP0 = 0, CBP1 = 64, RING = 192, YCOL = 256, TMEM_COLS = 512;
     static constexpr int EB = kI8 ? 1 : 2;
     static constexpr int C_BYTES = CROWS * kN * EB;
     static constexpr int B_BYTES = Q * kN * EB;
     static constexpr int H_BYTES = kP * kN * EB;
     static constexpr int NHB = kI8 ? 2 : 1;                      // state tile buffers
     static constexpr int X_BYTES = Q * 128;
-    static constexpr int PIECE = 128 * 128;                      // [128 rows][64 bf16]
-    static constexpr int RING_BYTES = kRing * PIECE;
     static constexpr int OFF_C = 0;
     static constexpr int OFF_B = C_BYTES;
-    // bf16: the ring reuses the B tile once CB is computed
-    static constexpr int OFF_RING = kI8 ? OFF_B + B_BYTES : OFF_B;
-    static constexpr int RB_END = kI8 ? OFF_RING + RING_BYTES : OFF_B + (B_BYTES > RING_BYTES ? B_BYTES : RING_BYTES);
-    static constexpr int OFF_X = (RB_END + 1023) & ~1023;
+    static constexpr int OFF_X = (OFF_B + B_BYTES + 1023) & ~1023;
     static constexpr int OFF_H = OFF_X + 2 * X_BYTES;
     static constexpr int OFF_VEC = OFF_H + NHB * H_BYTES;        // 2 slots x {acs, dtc, a2, vB, dtw}[Q]
     static constexpr int VEC_SLOT = 5 * Q * 4;
@@ -181,6 +181,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             tc::prefetch_tmap(&tm_b);
             tc::prefetch_tmap(&tm_c);
             tc::prefetch_tmap(&tm_h);
+            tc::prefetch_tmap(&tm_y);
             tc::mbar_arrive_expect_tx(bar + K::B_LOAD, K::C_BYTES + K::B_BYTES);
             if (!kI8) {
                 tc::tma_load_3d(sm + K::OFF_C, &tm_c, bar + K::B_LOAD, g * kN, c * Q, b);
@@ -214,33 +215,40 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // The issuing thread shares its SM sub-partition with busy CUDA-core warps, so
+        // every descriptor is precomputed and advanced by constant adds: an MMA costs a
+        // handful of instructions.  (Adding off >> 4 to a descriptor moves its start
+        // address by `off` bytes; addresses stay inside shared memory, so the 14-bit
+        // field never carries.)
         if (lane == 0) {
-            const uint32_t aC = tc::smem_u32(sm + K::OFF_C), aB = tc::smem_u32(sm + K::OFF_B);
-            const uint32_t aRing = tc::smem_u32(sm + K::OFF_RING);
             constexpr int kSteps = kI8 ? 4 : 8;                  // K = 128 (n)
-            auto descC = [&](int r0, int s) -> uint64_t {
-                const uint32_t off = kI8 ? (uint32_t)(s * 32) : (uint32_t)((s >> 2) * K::CROWS * 128 + (s & 3) * 32);
-                return tc::smem_desc(aC + r0 * 128 + off, 16, 1024, tc::kLayoutSw128);
-            };
-            auto descKm = [&](uint32_t base, int rows, int s) -> uint64_t {
-                const uint32_t off = kI8 ? (uint32_t)(s * 32) : (uint32_t)((s >> 2) * rows * 128 + (s & 3) * 32);
-                return tc::smem_desc(base + off, 16, 1024, tc::kLayoutSw128);
+            const uint64_t dC = tc::smem_desc(tc::smem_u32(sm + K::OFF_C), 16, 1024, tc::kLayoutSw128);
+            const uint64_t dB = tc::smem_desc(tc::smem_u32(sm + K::OFF_B), 16, 1024, tc::kLayoutSw128);
+            const uint64_t dH0 = tc::smem_desc(tc::smem_u32(sm + K::OFF_H), 16, 1024, tc::kLayoutSw128);
+            const uint64_t dX0 = tc::smem_desc(tc::smem_u32(sm + K::OFF_X), 0, 1024, tc::kLayoutSw128);
+            // byte offset of K step s inside a K-major tile whose 128-byte atoms hold `rows` rows
+            auto koff = [](int s, int rows) -> uint32_t {
+                return kI8 ? (uint32_t)(s * 32) : (uint32_t)((s >> 2) * rows * 128 + (s & 3) * 32);
             };
             bool ok = wait_bar(bar + K::B_LOAD, 0, abort_flag, status);
             if (ok) {
                 tc::tc_fence_after();
                 const uint32_t id0 = kI8 ? tc::idesc_s8_s32(128, K::NCB0, tc::kMajorK, tc::kMajorK)
                                          : tc::idesc_bf16_f32(128, K::NCB0, tc::kMajorK, tc::kMajorK);
-                for (int s = 0; s < kSteps; ++s) {
-                    if (kI8) tc::mma_i8_ss(tmem + K::CBF, descC(0, s), descKm(aB, Q, s), id0, s > 0);
-                    else tc::mma_f16_ss(tmem + K::CBF, descC(0, s), descKm(aB, Q, s), id0, s > 0);
+#pragma unroll
+                for (int st = 0; st < kSteps; ++st) {
+                    const uint64_t a = dC + (koff(st, K::CROWS) >> 4), bb = dB + (koff(st, Q) >> 4);
+                    if (kI8) tc::mma_i8_ss(tmem + K::CBF, a, bb, id0, st > 0);
+                    else tc::mma_f16_ss(tmem + K::CBF, a, bb, id0, st > 0);
                 }
                 if (K::JT == 2) {
                     const uint32_t id1 = kI8 ? tc::idesc_s8_s32(128, 256, tc::kMajorK, tc::kMajorK)
                                              : tc::idesc_bf16_f32(128, 256, tc::kMajorK, tc::kMajorK);
-                    for (int s = 0; s < kSteps; ++s) {
-                        if (kI8) tc::mma_i8_ss(tmem + K::CBF + 128, descC(128, s), descKm(aB, Q, s), id1, s > 0);
-                        else tc::mma_f16_ss(tmem + K::CBF + 128, descC(128, s), descKm(aB, Q, s), id1, s > 0);
+#pragma unroll
+                    for (int st = 0; st < kSteps; ++st) {
+                        const uint64_t a = dC + ((128 * 128 + koff(st, K::CROWS)) >> 4), bb = dB + (koff(st, Q) >> 4);
+                        if (kI8) tc::mma_i8_ss(tmem + K::CBF + 128, a, bb, id1, st > 0);
+                        else tc::mma_f16_ss(tmem + K::CBF + 128, a, bb, id1, st > 0);
                     }
                 }
                 tc::mma_commit(bar + K::B_CB);
@@ -260,17 +268,21 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 if (block) {
                     if (!wait_bar(bar + K::B_YEMPTY + s, (u & 1) ^ 1, abort_flag, status)) return false;
                     if (!wait_bar(bar + K::B_HFULL + hb, hpar, abort_flag, status)) return false;
-                } else if (!tc::mbar_try_wait(bar + K::B_YEMPTY + s, (u & 1) ^ 1) ||
-                           !tc::mbar_try_wait(bar + K::B_HFULL + hb, hpar)) {
+                } else if (!tc::mbar_test(bar + K::B_YEMPTY + s, (u & 1) ^ 1) ||
+                           !tc::mbar_test(bar + K::B_HFULL + hb, hpar)) {
                     return true;                                  // not yet: try again later
                 }
                 tc::tc_fence_after();
-                const uint32_t aH = tc::smem_u32(sm + K::OFF_H + hb * K::H_BYTES);
+                const uint64_t dH = dH0 + (uint64_t)((hb * K::H_BYTES) >> 4);
                 const uint32_t ycol = tmem + K::YCOL + 128 * s;
+#pragma unroll
                 for (int J = 0; J < K::JT; ++J)
+#pragma unroll
                     for (int st = 0; st < kSteps; ++st) {
-                        if (kI8) tc::mma_i8_ss(ycol + 64 * J, descC(128 * J, st), descKm(aH, kP, st), id_o, st > 0);
-                        else tc::mma_f16_ss(ycol + 64 * J, descC(128 * J, st), descKm(aH, kP, st), id_o, st > 0);
+                        const uint64_t a = dC + ((J * 128 * 128 + koff(st, K::CROWS)) >> 4);
+                        const uint64_t bb = dH + (koff(st, kP) >> 4);
+                        if (kI8) tc::mma_i8_ss(ycol + 64 * J, a, bb, id_o, st > 0);
+                        else tc::mma_f16_ss(ycol + 64 * J, a, bb, id_o, st > 0);
                     }
                 tc::mma_commit(bar + K::B_YOFULL + s);
                 tc::mma_commit(bar + K::B_HEMPTY + hb);
@@ -283,33 +295,30 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 const uint32_t u = (uint32_t)(it >> 1);
                 if (yo == it && !(ok = issue_yo(true))) break;
                 // waiting for this head's scaling: meanwhile start the next head's ChunkScan1
-                while (!tc::mbar_try_wait(bar + K::B_YSCALED + s, u & 1)) {
+                while (!tc::mbar_test(bar + K::B_YSCALED + s, u & 1)) {
                     if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
                     if (*abort_flag) { ok = false; break; }
                 }
                 if (!ok || !(ok = wait_bar(bar + K::B_YSCALED + s, u & 1, abort_flag, status))) break;
                 if (!(ok = wait_bar(bar + K::B_XFULL + s, u & 1, abort_flag, status))) break;
-                const uint32_t aX = tc::smem_u32(sm + K::OFF_X + s * K::X_BYTES);
+                const uint64_t dX = dX0 + (uint64_t)((s * K::X_BYTES) >> 4);
                 const uint32_t ycol = tmem + K::YCOL + 128 * s;
                 for (int k = 0; k < K::NPIECE; ++k, ++p) {
                     int J, ib;
                     piece_of(Q, k, J, ib);
-                    const int slot = p % kRing;
+                    const int slot = p & (kRing - 1);
                     const uint32_t rpar = (uint32_t)((p / kRing) & 1);
-                    while (!tc::mbar_try_wait(bar + K::B_RFULL + slot, rpar)) {
+                    while (!tc::mbar_test(bar + K::B_RFULL + slot, rpar)) {
                         if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
                         if (*abort_flag) { ok = false; break; }
                     }
-                    if (!ok || !(ok = wait_bar(bar + K::B_RFULL + slot, rpar, abort_flag, status))) break;
+                    if (!ok) break;
                     tc::tc_fence_after();
-                    const uint32_t am = aRing + slot * K::PIECE;
+                    const uint32_t am = tmem + K::RING + slot * 32;      // 64 bf16 = 32 columns
+                    const uint64_t db = dX + (uint64_t)(ib * 512);        // x rows ib*64: 64*128 B >> 4
+                    const uint32_t dcol = ycol + 64 * J;
 #pragma unroll
-                    for (int st = 0; st < 4; ++st) {
-                        const uint64_t da = tc::smem_desc(am + st * 32, 16, 1024, tc::kLayoutSw128);
-                        const uint64_t db = tc::smem_desc(aX + (uint32_t)((ib * 64 + st * 16) * 128), 0, 1024,
-                                                          tc::kLayoutSw128);
-                        tc::mma_f16_ss(ycol + 64 * J, da, db, id_d, 1u);
-                    }
+                    for (int st = 0; st < 4; ++st) tc::mma_f16_ts(dcol, am + st * 8, db + st * 128, id_d, 1u);
                     tc::mma_commit(bar + K::B_REMPTY + slot);
                 }
                 if (!ok) break;
@@ -399,7 +408,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 const int jb = j >> 6;
                 const float aj = a2[jc];
                 const float uj = ib < jb ? ex2(fminf(aj - a2[64 * ib + 63], 0.f)) : 0.f;
-                uint8_t* dst = sm + K::OFF_RING + slot * K::PIECE + r * 128;
+                const uint32_t tdst = trow + K::RING + slot * 32;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {                  // 32 columns at a time
                     uint32_t v[16];
@@ -408,32 +417,39 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     const int i0 = ib * 64 + hf * 32;
                     uint32_t out[16];
                     if (ib < jb) {
-                        const float* vb = vB + i0;
+                        const float4* vb4 = reinterpret_cast<const float4*>(vB + i0);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            out[e] = pack_bf16(bf16lo(v[e]) * (uj * vb[2 * e]), bf16hi(v[e]) * (uj * vb[2 * e + 1]));
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            const float4 f = vb4[e4];
+                            out[2 * e4] = pack_bf16(bf16lo(v[2 * e4]) * (uj * f.x), bf16hi(v[2 * e4]) * (uj * f.y));
+                            out[2 * e4 + 1] =
+                                pack_bf16(bf16lo(v[2 * e4 + 1]) * (uj * f.z), bf16hi(v[2 * e4 + 1]) * (uj * f.w));
+                        }
                     } else if (ib == jb) {
+                        const float4* a4 = reinterpret_cast<const float4*>(a2 + i0);
+                        const float4* d4 = reinterpret_cast<const float4*>(dtw + i0);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int i = i0 + 2 * e;
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            const float4 av = a4[e4], dv = d4[e4];
+                            const int i = i0 + 4 * e4;
                             // masked entries (i > j) would have a positive exponent: clamp, then select
-                            const float e0 = ex2(fminf(aj - a2[i], 0.f)) * dtw[i];
-                            const float e1 = ex2(fminf(aj - a2[i + 1], 0.f)) * dtw[i + 1];
-                            out[e] = pack_bf16((i <= j) ? bf16lo(v[e]) * e0 : 0.f,
-                                               (i + 1 <= j) ? bf16hi(v[e]) * e1 : 0.f);
+                            const float e0 = ex2(fminf(aj - av.x, 0.f)) * dv.x;
+                            const float e1 = ex2(fminf(aj - av.y, 0.f)) * dv.y;
+                            const float e2 = ex2(fminf(aj - av.z, 0.f)) * dv.z;
+                            const float e3 = ex2(fminf(aj - av.w, 0.f)) * dv.w;
+                            out[2 * e4] = pack_bf16((i <= j) ? bf16lo(v[2 * e4]) * e0 : 0.f,
+                                                    (i + 1 <= j) ? bf16hi(v[2 * e4]) * e1 : 0.f);
+                            out[2 * e4 + 1] = pack_bf16((i + 2 <= j) ? bf16lo(v[2 * e4 + 1]) * e2 : 0.f,
+                                                        (i + 3 <= j) ? bf16hi(v[2 * e4 + 1]) * e3 : 0.f);
                         }
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) out[e] = 0u;
                     }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int chunk = hf * 4 + q;
-                        *reinterpret_cast<uint4*>(dst + ((chunk ^ (r & 7)) << 4)) =
-                            make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
-                    }
+                    tc::tmem_st16(tdst + hf * 16, out);
                 }
-                tc::fence_proxy_async_smem();
+                tc::tmem_wait_st();
+                tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar + K::B_RFULL + slot);
             }
@@ -493,7 +509,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         }
     } else {
         // ------------------------------------------------------------ storers
-        const int et = tid - kStoreWarp0 * 32;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -537,14 +552,14 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             if (lane == 0) tc::mbar_arrive(bar + K::B_YEMPTY + s);
             tc::fence_proxy_async_smem();
             tc::named_sync(kIdStore, kEpiThreads);
-            if (et == 0) {
+            if (warp == kStoreWarp0 && lane == 0) {
                 tc::tma_store_3d(&tm_y, xs, h * kP, c * Q, b);
                 tc::tma_store_commit();
                 tc::tma_store_wait_read0();
                 tc::mbar_arrive(bar + K::B_XEMPTY + s);
             }
         }
-        if (et == 0) tc::tma_store_wait0();
+        if (warp == kStoreWarp0 && lane == 0) tc::tma_store_wait0();
     }
     __syncwarp();
     tc::tc_fence_before();
