@@ -82,11 +82,18 @@ def measured_peaks():
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
 # capture, keyed by kernel name, with the sha1 of the kernel source it was taken on.
 # A kernel whose source changed since reports null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # batch-2 capture scaled x4 to the batch-8 launch (traffic grows with the batch);
+    # see profiles/chunk_scan_tc_mamba2-2.7b-b2.md
+    ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.598528e6 + 127.595520e6),
+                                            "src_sha1": "a9cc8070ba81395147f80018bc89865f1ab66720"},
+    ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (271.073536e6 + 130.864896e6),
+                                            "src_sha1": "a9cc8070ba81395147f80018bc89865f1ab66720"},
+}
 
 
 def _src_hash(kernel: str):
-    f = {"chunk_scan": "chunk_scan.cu", "chunk_state": "chunk_state.cu", "state_passing": "state_passing.cu",
+    f = {"chunk_scan": "chunk_scan_tc.cu", "chunk_state": "chunk_state_tc.cu", "state_passing": "state_passing.cu",
          "chunk_cumsum": "cumsum.cu", "quantize_inputs": "quantize.cu"}.get(kernel)
     if not f:
         return None
