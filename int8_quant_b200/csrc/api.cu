@@ -59,7 +59,7 @@ T* at(void* base, size_t off) { return reinterpret_cast<T*>(reinterpret_cast<cha
 
 }  // namespace
 
-WsLayout ws_layout(const Dims& d, bool i8) {
+WsLayout ws_layout(const Dims& d, bool i8, bool fp32_states) {
     WsLayout w{};
     const size_t chains = (size_t)d.B * d.H;
     const size_t states = (size_t)d.B * d.nc * d.H * d.P * d.N;
@@ -69,7 +69,9 @@ WsLayout ws_layout(const Dims& d, bool i8) {
     w.lut = off;     off += align256(chains * d.nc * d.Q * sizeof(float));   // LUT_state
     w.dtc = off;     off += align256(chains * d.nc * d.Q * sizeof(float));   // dt, chunk-major
     w.decay = off;   off += align256(chains * d.nc * sizeof(float));   // fp32 decay or int32 code
-    w.states = off;  off += align256(states * (i8 ? 1 : sizeof(float)));
+    // chunk states: int8 (W8A8), bf16 (tensor-core bf16 path), fp32 (CUDA-core path, calibration)
+    const size_t s_elem = i8 ? 1 : (fp32_states || !tensor_core_shape(d)) ? sizeof(float) : sizeof(uint16_t);
+    w.states = off;  off += align256(states * s_elem);
     w.passed = off;  off += align256(states * (i8 ? 1 : sizeof(uint16_t)));
     w.total = off;
     return w;
@@ -203,17 +205,21 @@ ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const fl
     }
     float* Acs = at<float>(workspace, w.acs);
     float* decay = at<float>(workspace, w.decay);
-    float* S = at<float>(workspace, w.states);
     uint16_t* Hc = at<uint16_t>(workspace, w.passed);
     float* lut = at<float>(workspace, w.lut);
     float* dtc = at<float>(workspace, w.dtc);
     int* status = at<int>(workspace, w.status);
     SSD_STAGE("chunk_cumsum", launch_cumsum(d, dt, A, Acs, decay, nullptr, 0, status, lut, dtc, stream));
-    if (tensor_core_shape(d))
-        SSD_STAGE("chunk_state", launch_chunk_state_tc(d, false, x, B, lut, I8Scales{}, S, nullptr, nullptr, status, stream));
+    // bf16 chunk states on the tensor-core path, fp32 on the CUDA-core (small-shape) path
+    const bool tcs = tensor_core_shape(d);
+    void* S = at<void>(workspace, w.states);
+    if (tcs)
+        SSD_STAGE("chunk_state", launch_chunk_state_tc(d, false, x, B, lut, I8Scales{}, static_cast<uint16_t*>(S),
+                                                       nullptr, nullptr, status, stream));
     else
-        SSD_STAGE("chunk_state", launch_chunk_state_bf16(d, x, dt, Acs, B, S, nullptr, nullptr, stream));
-    SSD_STAGE("state_passing", launch_state_passing_bf16(d, S, decay, Hc, final_state, nullptr, stream));
+        SSD_STAGE("chunk_state", launch_chunk_state_bf16(d, x, dt, Acs, B, static_cast<float*>(S), nullptr, nullptr,
+                                                         stream));
+    SSD_STAGE("state_passing", launch_state_passing_bf16(d, S, !tcs, decay, Hc, final_state, nullptr, stream));
     if (tensor_core_shape(d))
         SSD_STAGE("chunk_scan", launch_chunk_scan_tc(d, false, x, B, C, Acs, dtc, D, I8Scales{}, Hc, y, nullptr,
                                                      kHeadsPerScanCta, status, stream));
@@ -281,7 +287,7 @@ ssd_status ssd_scan_fwd_i8(const ssd_shape* shape, const uint16_t* x, const floa
 }
 
 static WsLayout calib_layout(const Dims& p, size_t* fin_off, size_t* amax_off) {
-    WsLayout w = ws_layout(p, false);
+    WsLayout w = ws_layout(p, false, true);
     *fin_off = w.total;
     *amax_off = *fin_off + align256((size_t)p.B * p.H * p.P * p.N * sizeof(float));
     w.total = *amax_off + align256((size_t)(2 * p.G + 3 * p.H * p.P) * sizeof(float));
@@ -334,7 +340,7 @@ ssd_status ssd_calibrate_i8(const ssd_shape* shape, int prefix, const uint16_t* 
         SSD_TRY(launch_amax_bc(p, B, C, aB, aC, stream));
         SSD_TRY(launch_cumsum(p, dt, A, Acs, decay, nullptr, 0, nullptr, nullptr, nullptr, stream));
         SSD_TRY(launch_chunk_state_bf16(p, x, dt, Acs, B, S, ax, as, stream));
-        SSD_TRY(launch_state_passing_bf16(p, S, decay, nullptr, fin, ah, stream));
+        SSD_TRY(launch_state_passing_bf16(p, S, true, decay, nullptr, fin, ah, stream));
     }
     SSD_TRY(launch_amax_to_scale(aB, 2 * d.G + d.H * d.P, stream));       // s_B, s_C, s_x
     SSD_TRY(launch_amax_pair_to_scale(as, ah, s_s, d.H * d.P, stream));    // s_s over S and H

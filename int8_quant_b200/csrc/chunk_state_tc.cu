@@ -44,7 +44,7 @@ struct StateSmem {
 template <int Q, bool kI8>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                      Dims d, const float* __restrict__ lut_g, I8Scales sc, float* __restrict__ S,
+                      Dims d, const float* __restrict__ lut_g, I8Scales sc, uint16_t* __restrict__ S,
                       int8_t* __restrict__ S8, I8Debug dbg, int* __restrict__ status) {
     using L = StateSmem<Q, kI8>;
     extern __shared__ uint8_t smem_raw[];
@@ -170,7 +170,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
         for (int p = 0; p < kP; ++p) {
             const uint32_t raw = p < 32 ? v0[p] : v1[p - 32];
             if (!kI8) {
-                S[base + p * kN] = __uint_as_float(raw);
+                S[base + p * kN] = float_to_bf16_bits(__uint_as_float(raw));
             } else {
                 const int acc = (int)raw;
                 float q = rintf(__fmul_rn(__int2float_rn(acc), Mq[p]));
@@ -193,7 +193,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
 
 template <int Q, bool kI8>
 cudaError_t launch_q(const Dims& d, const CUtensorMap& tx, const CUtensorMap& tb, const float* lut,
-                     const I8Scales& sc, float* S, int8_t* S8, const I8Debug* dbg, int* status, cudaStream_t st) {
+                     const I8Scales& sc, uint16_t* S, int8_t* S8, const I8Debug* dbg, int* status, cudaStream_t st) {
     using L = StateSmem<Q, kI8>;
     auto k = chunk_state_tc_kernel<Q, kI8>;
     const int smem = L::kBytes + 1024;
@@ -207,7 +207,7 @@ cudaError_t launch_q(const Dims& d, const CUtensorMap& tx, const CUtensorMap& tb
 }  // namespace
 
 cudaError_t launch_chunk_state_tc(const Dims& d, bool i8, const uint16_t* x, const void* Bmat,
-                                  const float* lut, const I8Scales& sc, float* S, int8_t* S8,
+                                  const float* lut, const I8Scales& sc, uint16_t* S, int8_t* S8,
                                   const I8Debug* dbg, int* status, cudaStream_t st) {
     if (d.B == 0 || d.nc == 0) return cudaSuccess;
     if (d.P != kP || d.N != kN) return cudaErrorInvalidValue;

@@ -13,7 +13,8 @@ namespace ssd {
 struct WsLayout {
     size_t status, acs, lut, dtc, decay, states, passed, total;
 };
-WsLayout ws_layout(const Dims& d, bool i8);
+// `fp32_states`: chunk states kept in fp32 (calibration) instead of bf16 / int8.
+WsLayout ws_layout(const Dims& d, bool i8, bool fp32_states = false);
 
 // Optional W8A8 intermediates (device pointers, any may be null).
 struct I8Debug {
@@ -61,7 +62,7 @@ cudaError_t launch_chunk_state_i8(const Dims& d, const uint16_t* x, const float*
 //   bf16: H_{c+1} = decay_c * H_c + S_c in fp32; writes the state entering each
 //         chunk as bf16 (Hc) and/or fp32 (Hc32), the final state as fp32.
 //   W8A8: H_{c+1} = sat127(S8_c + ((dq_c * H_c + 2^(k-1)) >> k)).
-cudaError_t launch_state_passing_bf16(const Dims& d, const float* S, const float* decay,
+cudaError_t launch_state_passing_bf16(const Dims& d, const void* S, bool s_fp32, const float* decay,
                                       uint16_t* Hc, float* final_state, float* amax_h,
                                       cudaStream_t st);
 cudaError_t launch_state_passing_i8(const Dims& d, const int8_t* S8, const int32_t* dq, int shift,
@@ -98,8 +99,9 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, bool i8, const uint16_t* x, cons
 // Tensor-core ChunkState for P = 64, N = 128: one CTA per (head, chunk, batch row)
 // computes the chunk state transposed, S^T[n,p] = sum_j B[j,n] X_scaled[j,p], with
 // tcgen05 (kind::f16, or kind::i8 on Xq and Bq).  `lut` is LUT_state [B,H,nc,Q].
+// bf16 path: S written as bf16 (the passing accumulates in fp32).
 cudaError_t launch_chunk_state_tc(const Dims& d, bool i8, const uint16_t* x, const void* Bmat,
-                                  const float* lut, const I8Scales& sc, float* S, int8_t* S8,
+                                  const float* lut, const I8Scales& sc, uint16_t* S, int8_t* S8,
                                   const I8Debug* dbg, int* status, cudaStream_t st);
 
 // Calibration helpers.

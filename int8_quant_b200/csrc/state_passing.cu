@@ -1,5 +1,5 @@
 // state_passing.cu — a3, StatePassing (SSDi8 notes, eq. 6), sequential over chunks.
-//   bf16 : H_0 = 0, H_{c+1} = exp(Acs_c[Q-1]) * H_c + S_c               (fp32)
+//   bf16 : H_0 = 0, H_{c+1} = exp(Acs_c[Q-1]) * H_c + S_c  (fp32; S_c stored as bf16)
 //   W8A8 : H_{c+1} = sat127(S8_c + ((dq_c * H_c + 2^(k-1)) >> k))       (int32, then INT8)
 // Every (p,n) element of a (b,h) state is an independent scalar recurrence, so one
 // thread owns one element and walks the chunks; consecutive threads own consecutive
@@ -14,15 +14,20 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kAhead = 4;
 
+__device__ __forceinline__ float load_state(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float load_state(const uint16_t* p) { return bf16_bits_to_float(__ldg(p)); }
+
+// TS: element type of the chunk states (bf16 bits from the scan, fp32 for calibration).
+template <typename TS>
 __global__ void __launch_bounds__(kThreads)
-state_passing_bf16_kernel(Dims d, const float* __restrict__ S, const float* __restrict__ decay,
+state_passing_bf16_kernel(Dims d, const TS* __restrict__ S, const float* __restrict__ decay,
                           uint16_t* __restrict__ Hc, float* __restrict__ final_state, float* amax_h) {
     const int PN = d.P * d.N;
     const int e = blockIdx.x * kThreads + threadIdx.x;
     const int h = blockIdx.y, b = blockIdx.z;
     if (e >= PN) return;
     const long long stride = (long long)d.H * PN;                 // between chunks
-    const float* s = S + ((long long)b * d.nc * d.H + h) * PN + e;
+    const TS* s = S + ((long long)b * d.nc * d.H + h) * PN + e;
     uint16_t* hc = Hc ? Hc + ((long long)b * d.nc * d.H + h) * PN + e : nullptr;
     const float* dec = decay + ((long long)b * d.H + h) * d.nc;
     float hv = 0.f, amax = 0.f;
@@ -31,7 +36,7 @@ state_passing_bf16_kernel(Dims d, const float* __restrict__ S, const float* __re
 #pragma unroll
         for (int i = 0; i < kAhead; ++i) {
             const int c = c0 + i;
-            sv[i] = c < d.nc ? __ldg(s + c * stride) : 0.f;
+            sv[i] = c < d.nc ? load_state(s + c * stride) : 0.f;
             dv[i] = c < d.nc ? __ldg(dec + c) : 0.f;
         }
 #pragma unroll
@@ -83,12 +88,17 @@ state_passing_i8_kernel(Dims d, const int8_t* __restrict__ S8, const int32_t* __
 
 }  // namespace
 
-cudaError_t launch_state_passing_bf16(const Dims& d, const float* S, const float* decay,
+cudaError_t launch_state_passing_bf16(const Dims& d, const void* S, bool s_fp32, const float* decay,
                                       uint16_t* Hc, float* final_state, float* amax_h,
                                       cudaStream_t st) {
     if (d.B == 0) return cudaSuccess;
     dim3 grid((d.P * d.N + kThreads - 1) / kThreads, d.H, d.B);
-    state_passing_bf16_kernel<<<grid, kThreads, 0, st>>>(d, S, decay, Hc, final_state, amax_h);
+    if (s_fp32)
+        state_passing_bf16_kernel<float><<<grid, kThreads, 0, st>>>(d, static_cast<const float*>(S), decay, Hc,
+                                                                     final_state, amax_h);
+    else
+        state_passing_bf16_kernel<uint16_t><<<grid, kThreads, 0, st>>>(d, static_cast<const uint16_t*>(S), decay,
+                                                                        Hc, final_state, amax_h);
     return cudaGetLastError();
 }
 
