@@ -73,6 +73,7 @@ WsLayout ws_layout(const Dims& d, bool i8, bool fp32_states) {
     const size_t s_elem = i8 ? 1 : (fp32_states || !tensor_core_shape(d)) ? sizeof(float) : sizeof(uint16_t);
     w.states = off;  off += align256(states * s_elem);
     w.passed = off;  off += align256(states * (i8 ? 1 : sizeof(uint16_t)));
+    w.scales = off;  off += align256(i8 ? (size_t)2 * d.H * d.P * sizeof(float) : 0);   // 1/s_x, s_x s_B / s_s
     w.total = off;
     return w;
 }
@@ -214,7 +215,7 @@ ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const fl
     const bool tcs = tensor_core_shape(d);
     void* S = at<void>(workspace, w.states);
     if (tcs)
-        SSD_STAGE("chunk_state", launch_chunk_state_tc(d, false, x, B, lut, I8Scales{}, static_cast<uint16_t*>(S),
+        SSD_STAGE("chunk_state", launch_chunk_state_tc(d, false, x, B, lut, nullptr, nullptr, static_cast<uint16_t*>(S),
                                                        nullptr, nullptr, status, stream));
     else
         SSD_STAGE("chunk_state", launch_chunk_state_bf16(d, x, dt, Acs, B, static_cast<float*>(S), nullptr, nullptr,
@@ -257,9 +258,12 @@ ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, cons
     float* lut = at<float>(workspace, w.lut);
     float* dtc = at<float>(workspace, w.dtc);
     int* status = at<int>(workspace, w.status);
-    SSD_STAGE("chunk_cumsum", launch_cumsum(d, dt, A, Acs, nullptr, dq, sc.shift, status, lut, dtc, stream));
+    float* inv_sx = at<float>(workspace, w.scales);
+    float* mq = inv_sx + d.H * d.P;
+    SSD_STAGE("chunk_cumsum", launch_cumsum(d, dt, A, Acs, nullptr, dq, sc.shift, status, lut, dtc, stream, &sc, inv_sx, mq));
     if (tensor_core_shape(d))
-        SSD_STAGE("chunk_state", launch_chunk_state_tc(d, true, x, Bq, lut, sc, nullptr, S8, dbg ? &dd : nullptr, status, stream));
+        SSD_STAGE("chunk_state", launch_chunk_state_tc(d, true, x, Bq, lut, inv_sx, mq, nullptr, S8, dbg ? &dd : nullptr,
+                                                       status, stream));
     else
         SSD_STAGE("chunk_state", launch_chunk_state_i8(d, x, dt, Acs, Bq, sc, S8, dbg ? &dd : nullptr, stream));
     SSD_STAGE("state_passing", launch_state_passing_i8(d, S8, dq, sc.shift, H8, final_state, stream));

@@ -31,9 +31,23 @@ template <bool kI8>
 __global__ void __launch_bounds__(kThreads)
 cumsum_kernel(Dims d, const float* __restrict__ dt, const float* __restrict__ A,
               float* __restrict__ Acs, float* __restrict__ decay, int32_t* __restrict__ dq,
-              int shift, int* __restrict__ status, float* __restrict__ lut, float* __restrict__ dtc) {
+              int shift, int* __restrict__ status, float* __restrict__ lut, float* __restrict__ dtc,
+              I8Scales sc, float* __restrict__ inv_sx, float* __restrict__ mq) {
     // this call's kernels record device-side errors in the workspace status word
     if (status && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) *status = kStatusOk;
+    // W8A8: per-(h,p) quantisation reciprocal 1/s_x and requantisation multiplier
+    // s_x s_B / s_s of this block of heads, for ChunkState
+    if (kI8 && inv_sx && blockIdx.x == 0 && blockIdx.z == 0) {
+        for (int idx = threadIdx.x; idx < kHeadsPerCta * d.P; idx += kThreads) {
+            const int h = blockIdx.y * kHeadsPerCta + idx / d.P;
+            if (h < d.H) {
+                const int o = h * d.P + idx % d.P;
+                const float sx = __ldg(sc.s_x + o);
+                inv_sx[o] = __frcp_rn(sx);
+                mq[o] = __fdiv_rn(__fmul_rn(sx, __ldg(sc.s_B + h / d.hpg)), __ldg(sc.s_s + o));
+            }
+        }
+    }
     extern __shared__ float smem[];
     const int Q = d.Q, ld = pad(Q);
     float* tile = smem;                             // [kHeadsPerCta][ld]  dt
@@ -111,16 +125,18 @@ cumsum_kernel(Dims d, const float* __restrict__ dt, const float* __restrict__ A,
 
 cudaError_t launch_cumsum(const Dims& d, const float* dt, const float* A, float* Acs,
                           float* decay, int32_t* dq, int shift, int* status, float* lut, float* dtc,
-                          cudaStream_t st) {
+                          cudaStream_t st, const I8Scales* sc, float* inv_sx, float* mq) {
     if (d.B == 0 || d.nc == 0) return cudaSuccess;
     dim3 grid(d.nc, (d.H + kHeadsPerCta - 1) / kHeadsPerCta, d.B);
     const size_t smem = (size_t)2 * kHeadsPerCta * (d.Q + d.Q / 32) * sizeof(float);
     if (dq) {
         cudaFuncSetAttribute(cumsum_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        cumsum_kernel<true><<<grid, kThreads, smem, st>>>(d, dt, A, Acs, decay, dq, shift, status, lut, dtc);
+        cumsum_kernel<true><<<grid, kThreads, smem, st>>>(d, dt, A, Acs, decay, dq, shift, status, lut, dtc,
+                                                          sc ? *sc : I8Scales{}, sc ? inv_sx : nullptr, mq);
     } else {
         cudaFuncSetAttribute(cumsum_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        cumsum_kernel<false><<<grid, kThreads, smem, st>>>(d, dt, A, Acs, decay, dq, shift, status, lut, dtc);
+        cumsum_kernel<false><<<grid, kThreads, smem, st>>>(d, dt, A, Acs, decay, dq, shift, status, lut, dtc,
+                                                           I8Scales{}, nullptr, nullptr);
     }
     return cudaGetLastError();
 }

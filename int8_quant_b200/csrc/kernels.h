@@ -11,7 +11,7 @@ namespace ssd {
 
 // Workspace layout of one scan call (offsets in bytes, 256-byte aligned regions).
 struct WsLayout {
-    size_t status, acs, lut, dtc, decay, states, passed, total;
+    size_t status, acs, lut, dtc, decay, states, passed, scales, total;
 };
 // `fp32_states`: chunk states kept in fp32 (calibration) instead of bf16 / int8.
 WsLayout ws_layout(const Dims& d, bool i8, bool fp32_states = false);
@@ -44,10 +44,12 @@ cudaError_t launch_quantize_bc(const Dims& d, const uint16_t* B, const uint16_t*
 // a1: ChunkCumsum.  Writes Acs [B,H,nc,Q]; the bf16 path also the chunk decay
 // exp(Acs[Q-1]) (fp32 [B,H,nc]); the W8A8 path the decay codes (int32 [B,H,nc]).
 // Clears the workspace status word `status` (may be null) for the call.  `lut`
-// (LUT_state) and `dtc` (dt) are optional [B,H,nc,Q] outputs.
+// (LUT_state) and `dtc` (dt) are optional [B,H,nc,Q] outputs.  W8A8 with `sc`: also
+// inv_sx = 1/s_x and mq = s_x s_B / s_s per (h,p) ([H*P] each).
 cudaError_t launch_cumsum(const Dims& d, const float* dt, const float* A, float* Acs,
                           float* decay, int32_t* dq, int shift, int* status, float* lut, float* dtc,
-                          cudaStream_t st);
+                          cudaStream_t st, const I8Scales* sc = nullptr, float* inv_sx = nullptr,
+                          float* mq = nullptr);
 
 // a2: ChunkState.  bf16: fp32 states [B,nc,H,P,N]; W8A8: INT8 states.
 // amax_xs / amax_s (calibration only): per-(h,p) running max of |X_scaled| and |S_c|.
@@ -100,8 +102,9 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, bool i8, const uint16_t* x, cons
 // computes the chunk state transposed, S^T[n,p] = sum_j B[j,n] X_scaled[j,p], with
 // tcgen05 (kind::f16, or kind::i8 on Xq and Bq).  `lut` is LUT_state [B,H,nc,Q].
 // bf16 path: S written as bf16 (the passing accumulates in fp32).
+// W8A8: `inv_sx` and `mq` are the per-(h,p) tables ChunkCumsum writes.
 cudaError_t launch_chunk_state_tc(const Dims& d, bool i8, const uint16_t* x, const void* Bmat,
-                                  const float* lut, const I8Scales& sc, uint16_t* S, int8_t* S8,
+                                  const float* lut, const float* inv_sx, const float* mq, uint16_t* S, int8_t* S8,
                                   const I8Debug* dbg, int* status, cudaStream_t st);
 
 // Calibration helpers.

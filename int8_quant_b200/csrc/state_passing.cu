@@ -2,9 +2,9 @@
 //   bf16 : H_0 = 0, H_{c+1} = exp(Acs_c[Q-1]) * H_c + S_c  (fp32; S_c stored as bf16)
 //   W8A8 : H_{c+1} = sat127(S8_c + ((dq_c * H_c + 2^(k-1)) >> k))       (int32, then INT8)
 // Every (p,n) element of a (b,h) state is an independent scalar recurrence, so one
-// thread owns one element and walks the chunks; consecutive threads own consecutive
-// elements (coalesced loads and stores).  Loads of the next chunks' S are issued
-// ahead of the dependent update.
+// thread owns 4 consecutive elements and walks the chunks; consecutive threads own
+// consecutive elements (coalesced vector loads and stores).  Loads of the next
+// kAhead chunks' S are issued ahead of the dependent updates.
 #include "kernels.h"
 
 namespace ssd {
@@ -12,10 +12,21 @@ namespace ssd {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kAhead = 4;
+constexpr int kVec = 4;                                  // elements per thread (P*N % 4 == 0)
+constexpr int kAhead = 8;
 
-__device__ __forceinline__ float load_state(const float* p) { return __ldg(p); }
-__device__ __forceinline__ float load_state(const uint16_t* p) { return bf16_bits_to_float(__ldg(p)); }
+struct F4 {
+    float v[4];
+};
+__device__ __forceinline__ F4 load4(const float* p) {
+    const float4 t = __ldg(reinterpret_cast<const float4*>(p));
+    return F4{{t.x, t.y, t.z, t.w}};
+}
+__device__ __forceinline__ F4 load4(const uint16_t* p) {
+    const uint2 t = __ldg(reinterpret_cast<const uint2*>(p));
+    return F4{{__uint_as_float(t.x << 16), __uint_as_float(t.x & 0xffff0000u), __uint_as_float(t.y << 16),
+               __uint_as_float(t.y & 0xffff0000u)}};
+}
 
 // TS: element type of the chunk states (bf16 bits from the scan, fp32 for calibration).
 template <typename TS>
@@ -23,41 +34,49 @@ __global__ void __launch_bounds__(kThreads)
 state_passing_bf16_kernel(Dims d, const TS* __restrict__ S, const float* __restrict__ decay,
                           uint16_t* __restrict__ Hc, float* __restrict__ final_state, float* amax_h) {
     const int PN = d.P * d.N;
-    const int e = blockIdx.x * kThreads + threadIdx.x;
+    const int e = (blockIdx.x * kThreads + threadIdx.x) * kVec;
     const int h = blockIdx.y, b = blockIdx.z;
     if (e >= PN) return;
     const long long stride = (long long)d.H * PN;                 // between chunks
     const TS* s = S + ((long long)b * d.nc * d.H + h) * PN + e;
     uint16_t* hc = Hc ? Hc + ((long long)b * d.nc * d.H + h) * PN + e : nullptr;
     const float* dec = decay + ((long long)b * d.H + h) * d.nc;
-    float hv = 0.f, amax = 0.f;
+    float hv[kVec] = {0.f, 0.f, 0.f, 0.f};
+    float amax = 0.f;
     for (int c0 = 0; c0 < d.nc; c0 += kAhead) {
-        float sv[kAhead], dv[kAhead];
+        F4 sv[kAhead];
+        float dv[kAhead];
 #pragma unroll
         for (int i = 0; i < kAhead; ++i) {
             const int c = c0 + i;
-            sv[i] = c < d.nc ? load_state(s + c * stride) : 0.f;
+            sv[i] = c < d.nc ? load4(s + c * stride) : F4{{0.f, 0.f, 0.f, 0.f}};
             dv[i] = c < d.nc ? __ldg(dec + c) : 0.f;
         }
 #pragma unroll
         for (int i = 0; i < kAhead; ++i) {
             const int c = c0 + i;
             if (c < d.nc) {
-                if (hc) hc[c * stride] = float_to_bf16_bits(hv);
-                hv = fmaf(dv[i], hv, sv[i]);
-                amax = fmaxf(amax, fabsf(hv));
+                if (hc)
+                    *reinterpret_cast<uint2*>(hc + c * stride) =
+                        make_uint2((uint32_t)float_to_bf16_bits(hv[0]) | ((uint32_t)float_to_bf16_bits(hv[1]) << 16),
+                                   (uint32_t)float_to_bf16_bits(hv[2]) | ((uint32_t)float_to_bf16_bits(hv[3]) << 16));
+#pragma unroll
+                for (int v = 0; v < kVec; ++v) {
+                    hv[v] = fmaf(dv[i], hv[v], sv[i].v[v]);
+                    amax = fmaxf(amax, fabsf(hv[v]));
+                }
             }
         }
     }
-    final_state[((long long)b * d.H + h) * PN + e] = hv;
-    if (amax_h) atomic_max_nonneg(amax_h + h * d.P + e / d.N, amax);
+    *reinterpret_cast<float4*>(final_state + ((long long)b * d.H + h) * PN + e) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+    if (amax_h) atomic_max_nonneg(amax_h + h * d.P + e / d.N, amax);  // the 4 elements share p
 }
 
 __global__ void __launch_bounds__(kThreads)
 state_passing_i8_kernel(Dims d, const int8_t* __restrict__ S8, const int32_t* __restrict__ dq,
                         int shift, int8_t* __restrict__ H8, int8_t* __restrict__ final_state) {
     const int PN = d.P * d.N;
-    const int e = blockIdx.x * kThreads + threadIdx.x;
+    const int e = (blockIdx.x * kThreads + threadIdx.x) * kVec;
     const int h = blockIdx.y, b = blockIdx.z;
     if (e >= PN) return;
     const long long stride = (long long)d.H * PN;
@@ -65,25 +84,34 @@ state_passing_i8_kernel(Dims d, const int8_t* __restrict__ S8, const int32_t* __
     int8_t* hc = H8 + ((long long)b * d.nc * d.H + h) * PN + e;
     const int32_t* q = dq + ((long long)b * d.H + h) * d.nc;
     const int half = 1 << (shift - 1);
-    int hv = 0;
+    int hv[kVec] = {0, 0, 0, 0};
+    auto pack = [](const int (&v)[kVec]) -> uint32_t {
+        return (uint32_t)(v[0] & 0xff) | ((uint32_t)(v[1] & 0xff) << 8) | ((uint32_t)(v[2] & 0xff) << 16) |
+               ((uint32_t)(v[3] & 0xff) << 24);
+    };
     for (int c0 = 0; c0 < d.nc; c0 += kAhead) {
-        int sv[kAhead], qv[kAhead];
+        uint32_t sv[kAhead];
+        int qv[kAhead];
 #pragma unroll
         for (int i = 0; i < kAhead; ++i) {
             const int c = c0 + i;
-            sv[i] = c < d.nc ? (int)s[c * stride] : 0;
+            sv[i] = c < d.nc ? __ldg(reinterpret_cast<const unsigned int*>(s + c * stride)) : 0u;
             qv[i] = c < d.nc ? __ldg(q + c) : 0;
         }
 #pragma unroll
         for (int i = 0; i < kAhead; ++i) {
             const int c = c0 + i;
             if (c < d.nc) {
-                hc[c * stride] = (int8_t)hv;
-                hv = sat127(sv[i] + ((qv[i] * hv + half) >> shift));
+                *reinterpret_cast<uint32_t*>(hc + c * stride) = pack(hv);
+#pragma unroll
+                for (int v = 0; v < kVec; ++v) {
+                    const int sc = (int)(int8_t)(sv[i] >> (8 * v));          // sign-extended code
+                    hv[v] = sat127(sc + ((qv[i] * hv[v] + half) >> shift));
+                }
             }
         }
     }
-    final_state[((long long)b * d.H + h) * PN + e] = (int8_t)hv;
+    *reinterpret_cast<uint32_t*>(final_state + ((long long)b * d.H + h) * PN + e) = pack(hv);
 }
 
 }  // namespace
@@ -92,7 +120,8 @@ cudaError_t launch_state_passing_bf16(const Dims& d, const void* S, bool s_fp32,
                                       uint16_t* Hc, float* final_state, float* amax_h,
                                       cudaStream_t st) {
     if (d.B == 0) return cudaSuccess;
-    dim3 grid((d.P * d.N + kThreads - 1) / kThreads, d.H, d.B);
+    if ((d.P * d.N) % kVec != 0 || d.N % kVec != 0) return cudaErrorInvalidValue;
+    dim3 grid((d.P * d.N / kVec + kThreads - 1) / kThreads, d.H, d.B);
     if (s_fp32)
         state_passing_bf16_kernel<float><<<grid, kThreads, 0, st>>>(d, static_cast<const float*>(S), decay, Hc,
                                                                      final_state, amax_h);
@@ -105,7 +134,8 @@ cudaError_t launch_state_passing_bf16(const Dims& d, const void* S, bool s_fp32,
 cudaError_t launch_state_passing_i8(const Dims& d, const int8_t* S8, const int32_t* dq, int shift,
                                     int8_t* H8, int8_t* final_state, cudaStream_t st) {
     if (d.B == 0) return cudaSuccess;
-    dim3 grid((d.P * d.N + kThreads - 1) / kThreads, d.H, d.B);
+    if ((d.P * d.N) % kVec != 0) return cudaErrorInvalidValue;
+    dim3 grid((d.P * d.N / kVec + kThreads - 1) / kThreads, d.H, d.B);
     state_passing_i8_kernel<<<grid, kThreads, 0, st>>>(d, S8, dq, shift, H8, final_state);
     return cudaGetLastError();
 }

@@ -77,6 +77,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
 // About two seconds at the B200 boost clock: far longer than any legitimate wait here.
 constexpr long long kWaitLimit = 4000000000LL;
 
+// Bounded wait of a warp-specialised kernel: gives up at once when another role has
+// raised the CTA's abort flag; on expiry raises it and records `timeout_code` in the
+// status word (if any).
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              int* status, int timeout_code) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimit) {
+            *abort_flag = 1;
+            if (status) atomicExch(status, timeout_code);
+            return false;
+        }
+    }
+    return true;
+}
+
 // ---------------------------------------------------------------- proxies and TMA
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -170,6 +187,17 @@ __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint
         "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
         : "memory");
+}
+// True in exactly one lane of the (fully active) warp.  Issuing from an elected lane
+// of a warp that runs the whole schedule keeps the schedule's values warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t p;
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, e;\n\t}"
+        : "=r"(p));
+    return p != 0;
 }
 // Arrive on `bar` once every tcgen05 operation this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
