@@ -20,14 +20,14 @@
 //               the slot is free, ahead of the previous head's remaining work, since
 //               the tensor pipe executes in order), then y += M x over the pieces of
 //               the masked matrix as they arrive.
-//   warps 2-9   builders, two sets of four (one warp per TMEM lane quarter):
-//               M[j,i] = CB[j,i] exp(Acs_j - Acs_i) dt_i, 64 columns per piece, into
-//               a 2-slot ring in TMEM (bf16 pairs), which the y += M x MMAs read as
-//               their A operand: M never touches shared memory, whose bandwidth
-//               (128 B/clk) the skinny N = 64 MMAs already saturate.  Below the 64-row
-//               diagonal blocks the decay factorises through the block boundary r:
-//               exp(Acs_j - Acs_r) * exp(Acs_r - Acs_i), both <= 1, so only the
-//               diagonal blocks take an exponential per element.
+//   warps 2-9   builders: M[j,i] = CB[j,i] exp(Acs_j - Acs_i) dt_i, 64 columns per
+//               piece, into a 2-slot ring in TMEM (bf16 pairs), which the y += M x
+//               MMAs read as their A operand: M never touches shared memory, whose
+//               bandwidth (128 B/clk) the skinny N = 64 MMAs already saturate.  All
+//               eight warps build each piece, one 32 x 32 block each.  Below the
+//               32-row diagonal blocks the decay factorises through the end r of the
+//               block's columns, exp(Acs_j - Acs_r) * exp(Acs_r - Acs_i), both <= 1, so
+//               only the diagonal blocks take an exponential per element.
 //   warps 10-13 scalers: ChunkScan1 rows times exp(Acs_j) in TMEM (W8A8: dequantise).
 //   warps 14-17 storers: y + D x, rounded to bf16 over the x tile, stored by TMA
 //               (a warp's rows are 10 KB apart in y, so stores from registers would
@@ -60,9 +60,11 @@ struct Cfg {
     static constexpr int CROWS = Q >= 128 ? Q : 128;             // C rows loaded (Q = 64: ghost rows)
     static constexpr int NCB0 = Q >= 128 ? 128 : Q;              // CB columns of tile 0
     static constexpr int NPIECE = JT == 2 ? 6 : NCB0 / 64;       // 64-column pieces of M per head
-    // TMEM columns: packed CB at [0, 192), M ring at [192, 256), y slots at 256 + 128 s;
-    // the fp32 CB accumulators use [128, ...) before they are packed
-    static constexpr uint32_t CBF = 128, CBP0 = 0, CBP1 = 64, RING = 192, YCOL = 256, TMEM_COLS = 512;
+    // TMEM columns: packed CB of tile 1 at [0, 128) and of tile 0 at [128, 192), the M
+    // ring at [192, 256), y slots at 256 + 128 s.  Before packing, the fp32 CB
+    // accumulators use [128, 256) (tile 0) and [256, 512) (tile 1); tile 0 is packed in
+    // place, each 32-column step writing over columns it has already read.
+    static constexpr uint32_t CBF = 128, CBP0 = 128, CBP1 = 0, RING = 192, YCOL = 256, TMEM_COLS = 512;
     static constexpr int EB = kI8 ? 1 : 2;
     static constexpr int C_BYTES = CROWS * kN * EB;
     static constexpr int B_BYTES = Q * kN * EB;
@@ -80,7 +82,7 @@ struct Cfg {
     static constexpr int B_LOAD = 0, B_CB = 1, B_PACKED = 2, B_XFULL = 3, B_XEMPTY = 5, B_HFULL = 7,
                          B_HEMPTY = 9, B_VFULL = 11, B_VEMPTY = 13, B_RFULL = 15, B_REMPTY = 15 + kRing,
                          B_YOFULL = 15 + 2 * kRing, B_YSCALED = B_YOFULL + 2, B_YFULL = B_YOFULL + 4,
-                         B_YEMPTY = B_YOFULL + 6, NBAR = B_YOFULL + 8;
+                         B_YEMPTY = B_YOFULL + 6, B_VPREP = B_YOFULL + 8, NBAR = B_YOFULL + 10;
     static constexpr int OFF_FLAG = OFF_BAR + NBAR * 8;
     static constexpr int OFF_TMEM = OFF_FLAG + 8;
     static constexpr int BYTES = OFF_TMEM + 8;
@@ -118,6 +120,20 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Two IEEE fp32 operations (round to nearest even) in one packed instruction.
+__device__ __forceinline__ void mul_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void sub_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -150,11 +166,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
     if (tid == 0) {
         for (int i = 0; i < K::NBAR; ++i) {
             uint32_t cnt = 1;
-            if (i == K::B_PACKED) cnt = 4;
+            if (i == K::B_PACKED) cnt = 8;
             if (i >= K::B_VEMPTY && i < K::B_VEMPTY + 2) cnt = 12;
-            if (i >= K::B_RFULL && i < K::B_RFULL + kRing) cnt = 4;
+            if (i >= K::B_RFULL && i < K::B_RFULL + kRing) cnt = 8;
             if (i >= K::B_YSCALED && i < K::B_YSCALED + 2) cnt = 4;
             if (i >= K::B_YEMPTY && i < K::B_YEMPTY + 2) cnt = 4;
+            if (i >= K::B_VPREP && i < K::B_VPREP + 2) cnt = 4;
             tc::mbar_init(bar + i, cnt);
         }
         *abort_flag = 0;
@@ -215,24 +232,30 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // The issuing thread shares its SM sub-partition with busy CUDA-core warps, so
-        // every descriptor is precomputed and advanced by constant adds: an MMA costs a
-        // handful of instructions.  (Adding off >> 4 to a descriptor moves its start
-        // address by `off` bytes; addresses stay inside shared memory, so the 14-bit
-        // field never carries.)
-        if (lane == 0) {
-            constexpr int kSteps = kI8 ? 4 : 8;                  // K = 128 (n)
-            const uint64_t dC = tc::smem_desc(tc::smem_u32(sm + K::OFF_C), 16, 1024, tc::kLayoutSw128);
-            const uint64_t dB = tc::smem_desc(tc::smem_u32(sm + K::OFF_B), 16, 1024, tc::kLayoutSw128);
-            const uint64_t dH0 = tc::smem_desc(tc::smem_u32(sm + K::OFF_H), 16, 1024, tc::kLayoutSw128);
-            const uint64_t dX0 = tc::smem_desc(tc::smem_u32(sm + K::OFF_X), 0, 1024, tc::kLayoutSw128);
-            // byte offset of K step s inside a K-major tile whose 128-byte atoms hold `rows` rows
-            auto koff = [](int s, int rows) -> uint32_t {
-                return kI8 ? (uint32_t)(s * 32) : (uint32_t)((s >> 2) * rows * 128 + (s & 3) * 32);
-            };
-            bool ok = wait_bar(bar + K::B_LOAD, 0, abort_flag, status);
-            if (ok) {
-                tc::tc_fence_after();
+        // The whole warp runs the schedule, so that its values stay warp-uniform, and
+        // one elected lane issues; every readiness test is made uniform with a vote.
+        // Descriptors are precomputed and advanced by constant adds.  (Adding off >> 4
+        // to a descriptor moves its start address by `off` bytes; addresses stay
+        // inside shared memory, so the 14-bit field never carries.)
+        constexpr int kSteps = kI8 ? 4 : 8;                      // K = 128 (n)
+        const uint64_t dC = tc::smem_desc(tc::smem_u32(sm + K::OFF_C), 16, 1024, tc::kLayoutSw128);
+        const uint64_t dB = tc::smem_desc(tc::smem_u32(sm + K::OFF_B), 16, 1024, tc::kLayoutSw128);
+        const uint64_t dH0 = tc::smem_desc(tc::smem_u32(sm + K::OFF_H), 16, 1024, tc::kLayoutSw128);
+        const uint64_t dX0 = tc::smem_desc(tc::smem_u32(sm + K::OFF_X), 0, 1024, tc::kLayoutSw128);
+        // byte offset of K step s inside a K-major tile whose 128-byte atoms hold `rows` rows
+        auto koff = [](int s, int rows) -> uint32_t {
+            return kI8 ? (uint32_t)(s * 32) : (uint32_t)((s >> 2) * rows * 128 + (s & 3) * 32);
+        };
+        auto wait_all = [&](int which, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, wait_bar(bar + which, parity, abort_flag, status));
+        };
+        auto ready = [&](int which, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, tc::mbar_test(bar + which, parity));
+        };
+        bool ok = wait_all(K::B_LOAD, 0);
+        if (ok) {
+            tc::tc_fence_after();
+            if (tc::elect_one()) {
                 const uint32_t id0 = kI8 ? tc::idesc_s8_s32(128, K::NCB0, tc::kMajorK, tc::kMajorK)
                                          : tc::idesc_bf16_f32(128, K::NCB0, tc::kMajorK, tc::kMajorK);
 #pragma unroll
@@ -252,27 +275,29 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     }
                 }
                 tc::mma_commit(bar + K::B_CB);
-                ok = wait_bar(bar + K::B_PACKED, 0, abort_flag, status);
             }
-            const uint32_t id_o = kI8 ? tc::idesc_s8_s32(128, kP, tc::kMajorK, tc::kMajorK)
-                                      : tc::idesc_bf16_f32(128, kP, tc::kMajorK, tc::kMajorK);
-            const uint32_t id_d = tc::idesc_bf16_f32(128, kP, tc::kMajorK, tc::kMajorMN);
-            // ChunkScan1 of head `yo` into slot yo & 1, once that slot and the state tile
-            // are ready; `block` waits for them, otherwise the call only checks.
-            int yo = 0;
-            auto issue_yo = [&](bool block) -> bool {
-                const int s = yo & 1;
-                const uint32_t u = (uint32_t)(yo >> 1);
-                const int hb = kI8 ? s : 0;
-                const uint32_t hpar = kI8 ? (u & 1) : ((uint32_t)yo & 1);
-                if (block) {
-                    if (!wait_bar(bar + K::B_YEMPTY + s, (u & 1) ^ 1, abort_flag, status)) return false;
-                    if (!wait_bar(bar + K::B_HFULL + hb, hpar, abort_flag, status)) return false;
-                } else if (!tc::mbar_test(bar + K::B_YEMPTY + s, (u & 1) ^ 1) ||
-                           !tc::mbar_test(bar + K::B_HFULL + hb, hpar)) {
-                    return true;                                  // not yet: try again later
-                }
-                tc::tc_fence_after();
+            __syncwarp();
+            ok = wait_all(K::B_PACKED, 0);
+        }
+        const uint32_t id_o = kI8 ? tc::idesc_s8_s32(128, kP, tc::kMajorK, tc::kMajorK)
+                                  : tc::idesc_bf16_f32(128, kP, tc::kMajorK, tc::kMajorK);
+        const uint32_t id_d = tc::idesc_bf16_f32(128, kP, tc::kMajorK, tc::kMajorMN);
+        // ChunkScan1 of head `yo` into slot yo & 1, once that slot and the state tile
+        // are ready; `block` waits for them, otherwise the call only checks.
+        int yo = 0;
+        auto issue_yo = [&](bool block) -> bool {
+            const int s = yo & 1;
+            const uint32_t u = (uint32_t)(yo >> 1);
+            const int hb = kI8 ? s : 0;
+            const uint32_t hpar = kI8 ? (u & 1) : ((uint32_t)yo & 1);
+            if (block) {
+                if (!wait_all(K::B_YEMPTY + s, (u & 1) ^ 1)) return false;
+                if (!wait_all(K::B_HFULL + hb, hpar)) return false;
+            } else if (!ready(K::B_YEMPTY + s, (u & 1) ^ 1) || !ready(K::B_HFULL + hb, hpar)) {
+                return true;                                      // not yet: try again later
+            }
+            tc::tc_fence_after();
+            if (tc::elect_one()) {
                 const uint64_t dH = dH0 + (uint64_t)((hb * K::H_BYTES) >> 4);
                 const uint32_t ycol = tmem + K::YCOL + 128 * s;
 #pragma unroll
@@ -286,34 +311,37 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     }
                 tc::mma_commit(bar + K::B_YOFULL + s);
                 tc::mma_commit(bar + K::B_HEMPTY + hb);
-                ++yo;
-                return true;
-            };
-            int p = 0;                                            // ring piece counter
-            for (int it = 0; ok && it < nh; ++it) {
-                const int s = it & 1;
-                const uint32_t u = (uint32_t)(it >> 1);
-                if (yo == it && !(ok = issue_yo(true))) break;
-                // waiting for this head's scaling: meanwhile start the next head's ChunkScan1
-                while (!tc::mbar_test(bar + K::B_YSCALED + s, u & 1)) {
+            }
+            __syncwarp();
+            ++yo;
+            return true;
+        };
+        int p = 0;                                                // ring piece counter
+        for (int it = 0; ok && it < nh; ++it) {
+            const int s = it & 1;
+            const uint32_t u = (uint32_t)(it >> 1);
+            if (yo == it && !(ok = issue_yo(true))) break;
+            // waiting for this head's scaling: meanwhile start the next head's ChunkScan1
+            while (!ready(K::B_YSCALED + s, u & 1)) {
+                if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
+                if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
+            }
+            if (!ok || !(ok = wait_all(K::B_YSCALED + s, u & 1))) break;
+            if (!(ok = wait_all(K::B_XFULL + s, u & 1))) break;
+            const uint64_t dX = dX0 + (uint64_t)((s * K::X_BYTES) >> 4);
+            const uint32_t ycol = tmem + K::YCOL + 128 * s;
+            for (int k = 0; k < K::NPIECE; ++k, ++p) {
+                int J, ib;
+                piece_of(Q, k, J, ib);
+                const int slot = p & (kRing - 1);
+                const uint32_t rpar = (uint32_t)((p / kRing) & 1);
+                while (!ready(K::B_RFULL + slot, rpar)) {
                     if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
-                    if (*abort_flag) { ok = false; break; }
+                    if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
                 }
-                if (!ok || !(ok = wait_bar(bar + K::B_YSCALED + s, u & 1, abort_flag, status))) break;
-                if (!(ok = wait_bar(bar + K::B_XFULL + s, u & 1, abort_flag, status))) break;
-                const uint64_t dX = dX0 + (uint64_t)((s * K::X_BYTES) >> 4);
-                const uint32_t ycol = tmem + K::YCOL + 128 * s;
-                for (int k = 0; k < K::NPIECE; ++k, ++p) {
-                    int J, ib;
-                    piece_of(Q, k, J, ib);
-                    const int slot = p & (kRing - 1);
-                    const uint32_t rpar = (uint32_t)((p / kRing) & 1);
-                    while (!tc::mbar_test(bar + K::B_RFULL + slot, rpar)) {
-                        if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
-                        if (*abort_flag) { ok = false; break; }
-                    }
-                    if (!ok) break;
-                    tc::tc_fence_after();
+                if (!ok) break;
+                tc::tc_fence_after();
+                if (tc::elect_one()) {
                     const uint32_t am = tmem + K::RING + slot * 32;      // 64 bf16 = 32 columns
                     const uint64_t db = dX + (uint64_t)(ib * 512);        // x rows ib*64: 64*128 B >> 4
                     const uint32_t dcol = ycol + 64 * J;
@@ -321,16 +349,17 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     for (int st = 0; st < 4; ++st) tc::mma_f16_ts(dcol, am + st * 8, db + st * 128, id_d, 1u);
                     tc::mma_commit(bar + K::B_REMPTY + slot);
                 }
-                if (!ok) break;
-                tc::mma_commit(bar + K::B_YFULL + s);
+                __syncwarp();
             }
+            if (!ok) break;
+            if (tc::elect_one()) tc::mma_commit(bar + K::B_YFULL + s);
+            __syncwarp();
         }
     } else if (warp < kScaleWarp0) {
         // ------------------------------------------------------------ builders
-        const int bt = tid - kBuilderWarp0 * 32;
         const int set = (warp - kBuilderWarp0) >> 2;
         const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;                    // row within a 128-row tile
+        const int rrow = quarter * 32 + lane;                 // row within a 128-row tile
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
         bool ok = tc::named_and(kIdBuild, kBuilderThreads, wait_bar(bar + K::B_CB, 0, abort_flag, status));
         tc::tc_fence_after();
@@ -338,7 +367,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             if (kI8 && dbg.cb && (blockIdx.x % ctas_per_group) == 0) {
                 for (int J = 0; J < K::JT; ++J) {
                     const int ncol = J == 0 ? K::NCB0 : 256;
-                    const int j = J * 128 + r;
+                    const int j = J * 128 + rrow;
                     for (int g32 = 0; g32 < ncol / 32; ++g32) {
                         uint32_t v[32];
                         tc::tmem_ld32(trow + K::CBF + (J == 0 ? 0 : 128) + g32 * 32, v);
@@ -351,8 +380,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     }
                 }
             }
-            // pack CB to bf16 pairs: tile 0 first (its fp32 source is then overwritten by tile 1)
-            for (int J = 0; J < K::JT; ++J) {
+        }
+        if (ok) {
+            // pack CB to bf16 pairs: tile 0 by set 0, tile 1 by set 1 (both in parallel;
+            // the destinations do not overlap the other set's source columns)
+            const int J = set;
+            if (J < K::JT) {
                 const int ncol = J == 0 ? K::NCB0 : 256;
                 for (int g32 = 0; g32 < ncol / 32; ++g32) {
                     uint32_t v[32], w[16];
@@ -374,86 +407,109 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         }
         ok = tc::named_and(kIdBuild, kBuilderThreads, ok && wait_bar(bar + K::B_PACKED, 0, abort_flag, status));
         tc::tc_fence_after();
+        // Every piece is built by all eight warps.  Warp (set, quarter) owns the 32
+        // rows of its TMEM lane quarter and, of the piece's four 16-column groups, the
+        // groups set and set + 2, i.e. columns [16 set, 16 set + 16) of each of the
+        // piece's two 32-column blocks (so that the diagonal blocks' work is shared by
+        // both warps of a quarter).  Per 32 x 32 block of M: below the diagonal the decay
+        // factorises through the end r of the block's columns,
+        // exp(Acs_j - Acs_r) * exp(Acs_r - Acs_i) (both <= 1); on the diagonal it takes
+        // one exponential per element; above it is zero.  The next piece's CB columns
+        // are loaded from TMEM while the current piece is computed.
+        const int c0 = 16 * set;                                  // first column within a block
         int p = 0;
         for (int it = 0; ok && it < nh; ++it) {
             const int s = it & 1;
             const uint32_t u = (uint32_t)(it >> 1);
-            ok = tc::named_and(kIdBuild, kBuilderThreads, wait_bar(bar + K::B_VFULL + s, u & 1, abort_flag, status));
+            // the scalers have prepared the head's decay vectors
+            ok = tc::named_and(kIdBuild, kBuilderThreads, wait_bar(bar + K::B_VPREP + s, u & 1, abort_flag, status));
             if (!ok) break;
-            const float* acs = vec(s, kAcs);
-            const float* dts = vec(s, kDtc);
-            float* a2 = vec(s, kA2);
-            float* vB = vec(s, kVB);
-            float* dtw = vec(s, kDtw);
-            if (bt < Q) {
-                a2[bt] = acs[bt] * kLog2e;
-                dtw[bt] = dts[bt] * sCB;
-            }
-            tc::named_sync(kIdBuild, kBuilderThreads);
-            if (bt < Q) {
-                const int rr = min(64 * (bt / 64) + 63, Q - 1);
-                vB[bt] = ex2(fminf(a2[rr] - a2[bt], 0.f)) * dtw[bt];
-            }
-            tc::named_sync(kIdBuild, kBuilderThreads);
-            for (int k = set; k < K::NPIECE; k += 2) {
+            const float* a2 = vec(s, kA2);
+            const float* v32 = vec(s, kVB);
+            const float* dtw = vec(s, kDtw);
+            auto cb_cols = [&](int k) -> uint32_t {
                 int J, ib;
                 piece_of(Q, k, J, ib);
+                return trow + (J == 0 ? K::CBP0 : K::CBP1) + ib * 32 + c0 / 2;
+            };
+            // one 16-column group of block `cb` (columns i0 + c0 .. i0 + c0 + 15)
+            auto build16 = [&](const uint32_t (&v)[8], int jb, int cb, float aj, uint32_t (&out)[8]) {
+                const int i0 = 32 * cb + c0;
+                if (jb > cb) {
+                    const float uj = ex2(fminf(aj - a2[32 * cb + 31], 0.f));
+                    const float4* v4 = reinterpret_cast<const float4*>(v32 + i0);
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const float4 f = v4[e4];
+                        float w0, w1, w2, w3, m0, m1, m2, m3;
+                        mul_f32x2(w0, w1, uj, uj, f.x, f.y);
+                        mul_f32x2(w2, w3, uj, uj, f.z, f.w);
+                        mul_f32x2(m0, m1, bf16lo(v[2 * e4]), bf16hi(v[2 * e4]), w0, w1);
+                        mul_f32x2(m2, m3, bf16lo(v[2 * e4 + 1]), bf16hi(v[2 * e4 + 1]), w2, w3);
+                        out[2 * e4] = pack_bf16(m0, m1);
+                        out[2 * e4 + 1] = pack_bf16(m2, m3);
+                    }
+                } else if (jb == cb) {
+                    // masked entries (column > row) have a positive exponent; they are
+                    // selected away, whatever the exponential gives
+                    const float4* a4 = reinterpret_cast<const float4*>(a2 + i0);
+                    const float4* d4 = reinterpret_cast<const float4*>(dtw + i0);
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const float4 av = a4[e4], dv = d4[e4];
+                        float x0, x1, x2, x3;
+                        sub_f32x2(x0, x1, aj, aj, av.x, av.y);
+                        sub_f32x2(x2, x3, aj, aj, av.z, av.w);
+                        float t0, t1, t2, t3, m0, m1, m2, m3;
+                        mul_f32x2(t0, t1, ex2(x0), ex2(x1), dv.x, dv.y);
+                        mul_f32x2(t2, t3, ex2(x2), ex2(x3), dv.z, dv.w);
+                        mul_f32x2(m0, m1, bf16lo(v[2 * e4]), bf16hi(v[2 * e4]), t0, t1);
+                        mul_f32x2(m2, m3, bf16lo(v[2 * e4 + 1]), bf16hi(v[2 * e4 + 1]), t2, t3);
+                        const int c = c0 + 4 * e4;                // column within the block; the row is `lane`
+                        out[2 * e4] = pack_bf16(c <= lane ? m0 : 0.f, c + 1 <= lane ? m1 : 0.f);
+                        out[2 * e4 + 1] = pack_bf16(c + 2 <= lane ? m2 : 0.f, c + 3 <= lane ? m3 : 0.f);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) out[e] = 0u;
+                }
+            };
+            uint32_t cbv[2][2][8];                                // [buffer][block of the piece][packed cols]
+            tc::tmem_ld8(cb_cols(0), cbv[0][0]);
+            tc::tmem_ld8(cb_cols(0) + 16, cbv[0][1]);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < K::NPIECE; ++k) {
+                int J, ib;
+                piece_of(Q, k, J, ib);
+                const bool pre = k + 1 < K::NPIECE;
+                if (pre) {
+                    tc::tmem_ld8(cb_cols(k + 1), cbv[(k + 1) & 1][0]);
+                    tc::tmem_ld8(cb_cols(k + 1) + 16, cbv[(k + 1) & 1][1]);
+                }
                 const int pp = p + k, slot = pp % kRing;
-                if (!wait_bar(bar + K::B_REMPTY + slot, (uint32_t)(((pp / kRing) & 1) ^ 1), abort_flag, status)) {
+                const int jrow = J * 128 + rrow;                  // row of M (ghost rows >= Q when Q = 64)
+                const int jb = 4 * J + quarter;                   // its 32-row block
+                const float aj = a2[jrow < Q ? jrow : Q - 1];
+                uint32_t out0[8], out1[8];
+                build16(cbv[k & 1][0], jb, 2 * ib, aj, out0);
+                build16(cbv[k & 1][1], jb, 2 * ib + 1, aj, out1);
+                if (!__all_sync(0xffffffffu, wait_bar(bar + K::B_REMPTY + slot, (uint32_t)(((pp / kRing) & 1) ^ 1),
+                                                      abort_flag, status))) {
                     ok = false;
                     break;
                 }
-                const int j = J * 128 + r;
-                const int jc = j < Q ? j : Q - 1;
-                const int jb = j >> 6;
-                const float aj = a2[jc];
-                const float uj = ib < jb ? ex2(fminf(aj - a2[64 * ib + 63], 0.f)) : 0.f;
-                const uint32_t tdst = trow + K::RING + slot * 32;
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {                  // 32 columns at a time
-                    uint32_t v[16];
-                    tc::tmem_ld16(trow + (J == 0 ? K::CBP0 : K::CBP1) + ib * 32 + hf * 16, v);
-                    tc::tmem_wait_ld();
-                    const int i0 = ib * 64 + hf * 32;
-                    uint32_t out[16];
-                    if (ib < jb) {
-                        const float4* vb4 = reinterpret_cast<const float4*>(vB + i0);
-#pragma unroll
-                        for (int e4 = 0; e4 < 8; ++e4) {
-                            const float4 f = vb4[e4];
-                            out[2 * e4] = pack_bf16(bf16lo(v[2 * e4]) * (uj * f.x), bf16hi(v[2 * e4]) * (uj * f.y));
-                            out[2 * e4 + 1] =
-                                pack_bf16(bf16lo(v[2 * e4 + 1]) * (uj * f.z), bf16hi(v[2 * e4 + 1]) * (uj * f.w));
-                        }
-                    } else if (ib == jb) {
-                        const float4* a4 = reinterpret_cast<const float4*>(a2 + i0);
-                        const float4* d4 = reinterpret_cast<const float4*>(dtw + i0);
-#pragma unroll
-                        for (int e4 = 0; e4 < 8; ++e4) {
-                            const float4 av = a4[e4], dv = d4[e4];
-                            const int i = i0 + 4 * e4;
-                            // masked entries (i > j) would have a positive exponent: clamp, then select
-                            const float e0 = ex2(fminf(aj - av.x, 0.f)) * dv.x;
-                            const float e1 = ex2(fminf(aj - av.y, 0.f)) * dv.y;
-                            const float e2 = ex2(fminf(aj - av.z, 0.f)) * dv.z;
-                            const float e3 = ex2(fminf(aj - av.w, 0.f)) * dv.w;
-                            out[2 * e4] = pack_bf16((i <= j) ? bf16lo(v[2 * e4]) * e0 : 0.f,
-                                                    (i + 1 <= j) ? bf16hi(v[2 * e4]) * e1 : 0.f);
-                            out[2 * e4 + 1] = pack_bf16((i + 2 <= j) ? bf16lo(v[2 * e4 + 1]) * e2 : 0.f,
-                                                        (i + 3 <= j) ? bf16hi(v[2 * e4 + 1]) * e3 : 0.f);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) out[e] = 0u;
-                    }
-                    tc::tmem_st16(tdst + hf * 16, out);
-                }
+                const uint32_t dst = trow + K::RING + slot * 32 + c0 / 2;
+                tc::tmem_st8(dst, out0);
+                tc::tmem_st8(dst + 16, out1);
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar + K::B_RFULL + slot);
+                if (pre) tc::tmem_wait_ld();
             }
-            // both sets leave together if either gave up
+            tc::tmem_wait_ld();                                   // no load left in flight on an early exit
+            // all builders leave together if any gave up
             ok = tc::named_and(kIdBuild, kBuilderThreads, ok);
             if (!ok) break;
             p += K::NPIECE;
@@ -469,9 +525,30 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         for (int it = 0; ok && it < nh; ++it) {
             const int h = h0 + it, s = it & 1;
             const uint32_t u = (uint32_t)(it >> 1);
-            bool w = wait_bar(bar + K::B_VFULL + s, u & 1, abort_flag, status);
-            w = w && wait_bar(bar + K::B_YOFULL + s, u & 1, abort_flag, status);
-            if (!(ok = tc::named_and(kIdScale, kEpiThreads, w))) break;
+            if (!(ok = tc::named_and(kIdScale, kEpiThreads, wait_bar(bar + K::B_VFULL + s, u & 1, abort_flag, status))))
+                break;
+            {
+                // the builders' decay vectors: log2-scaled Acs, dt with CB's
+                // dequantisation, and the column factor exp(Acs_r - Acs_i) dt_i towards
+                // the end r of i's 32-column block
+                const float* acs = vec(s, kAcs);
+                const float* dts = vec(s, kDtc);
+                float* a2 = vec(s, kA2);
+                float* v32 = vec(s, kVB);
+                float* dtw = vec(s, kDtw);
+                for (int i = tid - kScaleWarp0 * 32; i < Q; i += kEpiThreads) {
+                    const float ai = acs[i] * kLog2e;
+                    const float ar = acs[i | 31] * kLog2e;
+                    const float dw = dts[i] * sCB;
+                    a2[i] = ai;
+                    dtw[i] = dw;
+                    v32[i] = ex2(fminf(ar - ai, 0.f)) * dw;
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar + K::B_VPREP + s);
+            }
+            if (!(ok = tc::named_and(kIdScale, kEpiThreads, wait_bar(bar + K::B_YOFULL + s, u & 1, abort_flag, status))))
+                break;
             tc::tc_fence_after();
             const float* acs = vec(s, kAcs);
             const uint32_t ybase = trow + K::YCOL + 128 * s;
