@@ -53,20 +53,22 @@ def kernel_bytes(w, path: str, kernel: str) -> int:
     nc = w.nchunks
     chains = w.batch * H
     states = w.batch * nc * H * P * N
+    tc_shape = (P, N) == (64, 128)                              # tensor-core kernels
     bc = 1 if path == "w8a8" else 2                            # bytes per B/C element read by the scan
-    st_w = 1 if path == "w8a8" else 4                           # chunk-state element
+    st_w = 1 if path == "w8a8" else (2 if tc_shape else 4)     # chunk-state element
     hc_w = 1 if path == "w8a8" else 2                           # passed-state element
-    acs = chains * nc * Q * 4
+    vec = chains * nc * Q * 4                                   # one [B,H,nc,Q] fp32 vector (Acs, LUT_state, dt)
+    fin = w.batch * H * P * N * (4 if path == "bf16" else 1)
     if kernel == "quantize_inputs":
         return T * G * N * (2 * 2 + 2 * 1)
-    if kernel == "chunk_cumsum":
-        return T * H * 4 + acs + chains * nc * 4
-    if kernel == "chunk_state":
-        return T * (2 * H * P + bc * G * N + 4 * H) + acs + states * st_w
-    if kernel == "state_passing":
-        return states * st_w + chains * nc * 4 + states * hc_w + w.batch * H * P * N * (4 if path == "bf16" else 1)
-    if kernel == "chunk_scan":
-        return T * (2 * H * P + 2 * bc * G * N + 4 * H + 2 * H * P) + acs + states * hc_w
+    if kernel == "chunk_cumsum":                                # dt in; Acs, LUT_state, dt chunk-major, decay out
+        return T * H * 4 + 3 * vec + chains * nc * 4
+    if kernel == "chunk_state":                                 # x, B, LUT_state in; chunk states out
+        return T * (2 * H * P + bc * G * N) + vec + states * st_w
+    if kernel == "state_passing":                               # states, decay in; passed states, final out
+        return states * st_w + chains * nc * 4 + states * hc_w + fin
+    if kernel == "chunk_scan":                                  # x, B, C, Acs, dt, passed states in; y out
+        return T * (2 * H * P + 2 * bc * G * N + 2 * H * P) + 2 * vec + states * hc_w
     return 0
 
 
@@ -85,10 +87,10 @@ def measured_peaks():
 NCU_TRAFFIC = {
     # batch-2 capture scaled x4 to the batch-8 launch (traffic grows with the batch);
     # see profiles/chunk_scan_tc_mamba2-2.7b-b2.md
-    ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.598528e6 + 127.595520e6),
-                                            "src_sha1": "a9cc8070ba81395147f80018bc89865f1ab66720"},
-    ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (271.073536e6 + 130.864896e6),
-                                            "src_sha1": "a9cc8070ba81395147f80018bc89865f1ab66720"},
+    ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.653312e6 + 129.440512e6),
+                                            "src_sha1": "37e9f4c1cc4b22536816c1e3d85d4e6bd2f95fcc"},
+    ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (270.715648e6 + 130.753280e6),
+                                            "src_sha1": "37e9f4c1cc4b22536816c1e3d85d4e6bd2f95fcc"},
 }
 
 
@@ -223,6 +225,23 @@ def cpu_oracle_sample(w, path: str, budget_s: float, pool=None):
 
 
 # ---------------------------------------------------------------- GPU arm
+# ---------------------------------------------------------------- replicas
+def max_over_ranks(v: float, dist=None, device="cpu") -> float:
+    """The largest of every rank's `v` (the slowest replica's time); `dist` None: one process."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(tokens_per_rank: int, ms_per_step: float, world: int) -> float:
+    """Whole-job tokens/s of `world` replicas that each process `tokens_per_rank` tokens per step,
+    with the step time taken as the max over ranks (weak scaling)."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def run_ours(args, rank, world, dist):
     import torch
     import int8_quant_b200 as iq
@@ -249,13 +268,6 @@ def run_ours(args, rank, world, dist):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     def timed(path):
         step = step_fn(path)
         for _ in range(args.warmup):
@@ -274,7 +286,7 @@ def run_ours(args, rank, world, dist):
             torch.cuda.synchronize()
             iq.ssd_profile_enable(False)
             barrier()
-        ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.steps
+        ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev) / args.steps
         kern = iq.ssd_profile_read()
         return ms, kern, clk.summary()
 
@@ -315,8 +327,8 @@ def run_ours(args, rank, world, dist):
             ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms = max_over_ranks(ev0.elapsed_time(ev1)) / n
-        return {"value": world * w.tokens / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev) / n
+        return {"value": replica_throughput(w.tokens, ms, world), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4), "steps": n}
 
     results = {}
@@ -326,7 +338,7 @@ def run_ours(args, rank, world, dist):
         launches = sum(c for _, c in kern.values())
         alg = path_bytes(w, path)
         results[path] = {
-            "ms_per_step": ms, "value": world * w.tokens / (ms / 1e3), "kern": kern, "clocks": clocks,
+            "ms_per_step": ms, "value": replica_throughput(w.tokens, ms, world), "kern": kern, "clocks": clocks,
             "roofline": roofline(path, kern), "gpu_launches": launches,
             "path_roofline": {"alg_bytes": alg, "achieved_GBs": round(alg / (ms / 1e3) / 1e9, 1),
                               "frac_of_measured_hbm": round(alg / (ms / 1e3) / 1e9 / peak, 4),
