@@ -84,6 +84,10 @@ typedef struct {
 /* Human-readable name of a status code (static string). */
 const char* ssd_status_string(ssd_status s);
 
+/* The CUDA runtime's message for the error behind the calling thread's most recent
+ * SSD_ERR_CUDA ("no error" if there was none); a static string. */
+const char* ssd_last_cuda_error(void);
+
 /* Bytes of device workspace that ssd_scan_fwd_bf16 (is_i8 = 0) or ssd_scan_fwd_i8
  * (is_i8 = 1) need for `shape`; 0 for an invalid or unsupported shape.  The
  * workspace holds the per-chunk cumulative decays, chunk states and passed states

@@ -46,12 +46,19 @@ bool tensor_core_shape(const Dims& d) { return d.P == 64 && d.N == 128; }
 // Heads that share one ChunkBMM result in the tensor-core ChunkScan.
 constexpr int kHeadsPerScanCta = 8;
 
-ssd_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
+// The CUDA error behind this thread's last SSD_ERR_CUDA (cudaSuccess if none).
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+ssd_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return SSD_OK;
+    g_last_cuda_error = e;
+    return SSD_ERR_CUDA;
+}
 
 #define SSD_TRY(expr)                                  \
     do {                                               \
         cudaError_t _e = (expr);                       \
-        if (_e != cudaSuccess) return SSD_ERR_CUDA;    \
+        if (_e != cudaSuccess) return from_cuda(_e);   \
     } while (0)
 
 template <typename T>
@@ -132,7 +139,7 @@ struct Scope {
     do {                                                           \
         prof::Scope _scope(name, stream);                          \
         cudaError_t _e = (expr);                                   \
-        if (_e != cudaSuccess) return SSD_ERR_CUDA;                \
+        if (_e != cudaSuccess) return from_cuda(_e);               \
     } while (0)
 
 }  // namespace ssd
@@ -152,6 +159,8 @@ const char* ssd_status_string(ssd_status s) {
     }
     return "unknown ssd_status";
 }
+
+const char* ssd_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 size_t ssd_workspace_bytes(const ssd_shape* shape, int is_i8) {
     Dims d;

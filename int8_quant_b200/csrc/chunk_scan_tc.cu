@@ -422,7 +422,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             const int s = it & 1;
             const uint32_t u = (uint32_t)(it >> 1);
             // the scalers have prepared the head's decay vectors
-            ok = tc::named_and(kIdBuild, kBuilderThreads, wait_bar(bar + K::B_VPREP + s, u & 1, abort_flag, status));
+            ok = __all_sync(0xffffffffu, wait_bar(bar + K::B_VPREP + s, u & 1, abort_flag, status));
             if (!ok) break;
             const float* a2 = vec(s, kA2);
             const float* v32 = vec(s, kVB);
@@ -509,8 +509,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 if (pre) tc::tmem_wait_ld();
             }
             tc::tmem_wait_ld();                                   // no load left in flight on an early exit
-            // all builders leave together if any gave up
-            ok = tc::named_and(kIdBuild, kBuilderThreads, ok);
             if (!ok) break;
             p += K::NPIECE;
             __syncwarp();

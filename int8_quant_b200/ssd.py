@@ -18,7 +18,7 @@ STATUS_NAMES = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
                 4: "SSD_ERR_CUDA", 5: "SSD_ERR_TIMEOUT"}
 
 # Names declared in include/ssd.h (checked against the header by the tests).
-EXPORTS = ("ssd_status_string", "ssd_workspace_bytes", "ssd_quantize_inputs", "ssd_scan_fwd_bf16",
+EXPORTS = ("ssd_status_string", "ssd_last_cuda_error", "ssd_workspace_bytes", "ssd_quantize_inputs", "ssd_scan_fwd_bf16",
            "ssd_scan_fwd_i8", "ssd_scan_fwd_i8_debug", "ssd_calibrate_workspace_bytes",
            "ssd_calibrate_i8", "ssd_workspace_status", "ssd_profile_enable", "ssd_profile_read",
            "ssd_profile_reset", "ssd_scan_fwd_bf16_static")
@@ -52,7 +52,10 @@ class SsdI8Debug(ctypes.Structure):
 class SsdError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = int(status)
-        super().__init__(f"{fn}: {_lib().ssd_status_string(status).decode()}")
+        msg = f"{fn}: {_lib().ssd_status_string(status).decode()}"
+        if status == 4:  # SSD_ERR_CUDA
+            msg += f" ({_lib().ssd_last_cuda_error().decode()})"
+        super().__init__(msg)
 
 
 _LIB = None
@@ -68,6 +71,8 @@ def _lib():
         sp = ctypes.POINTER(SsdShape)
         lib.ssd_status_string.restype = ctypes.c_char_p
         lib.ssd_status_string.argtypes = [I]
+        lib.ssd_last_cuda_error.restype = ctypes.c_char_p
+        lib.ssd_last_cuda_error.argtypes = []
         lib.ssd_workspace_bytes.restype = S
         lib.ssd_workspace_bytes.argtypes = [sp, I]
         lib.ssd_calibrate_workspace_bytes.restype = S
