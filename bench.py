@@ -304,32 +304,32 @@ def run_ours(args, rank, world, dist):
                 "kernel_shares": {k: round(v[0] / sum(x[0] for x in kern.values()), 4) for k, v in kern.items()}}
 
     def e2e(path):
-        """Same metric with host buffers: pinned H2D of the step's inputs, the call, D2H of the outputs."""
-        step = step_fn(path)
+        """Same metric with the batch in pinned host memory: every step copies the inputs in and y and
+        the final state out, group by group (StreamedScan), overlapping the copies with the scans."""
+        from int8_quant_b200.runner import StreamedScan
         names = ["x", "dt", "B", "C"]
-        hbufs = {k: dinp[k].to("cpu").pin_memory() for k in names}
-        out_dev = [pb.y, pb.final8 if path == "w8a8" else pb.final32]
-        out_host = [torch.empty_like(t, device="cpu").pin_memory() for t in out_dev]
-        h2d = sum(t.numel() * t.element_size() for t in hbufs.values())
-        d2h = sum(t.numel() * t.element_size() for t in out_host)
+        host_io = {k: dinp[k].to("cpu").pin_memory() for k in names}
+        fin = pb.final8 if path == "w8a8" else pb.final32
+        host_io["y"] = torch.empty_like(pb.y, device="cpu").pin_memory()
+        host_io["final"] = torch.empty_like(fin, device="cpu").pin_memory()
+        runner = StreamedScan(host_io, dinp["A"], dinp["D"], w.chunk, path, rows_per_group=1,
+                              scales=pb.scales if path == "w8a8" else None, device=dev)
         n = max(1, min(args.steps, args.e2e_steps))
+        runner.run()                                             # warm-up
+        torch.cuda.synchronize()
+        barrier()
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            for i in range(n + 1):
-                if i == 1:
-                    barrier()
-                    ev0.record(stream)
-                for k in names:
-                    dinp[k].copy_(hbufs[k], non_blocking=True)
-                step()
-                for dsrc, hdst in zip(out_dev, out_host):
-                    hdst.copy_(dsrc, non_blocking=True)
-            ev1.record(stream)
+        ev0.record(runner.streams[0])
+        for _ in range(n):
+            runner.run()
+        ev1.record(runner.streams[2])
         torch.cuda.synchronize()
         barrier()
         ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev) / n
-        return {"value": replica_throughput(w.tokens, ms, world), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4), "steps": n}
+        return {"value": replica_throughput(w.tokens, ms, world), "unit": "tokens/s",
+                "h2d_bytes_per_step": runner.h2d_bytes, "d2h_bytes_per_step": runner.d2h_bytes,
+                "ms_per_step": round(ms, 4), "steps": n, "rows_per_group": 1,
+                "api": "ssd_quantize_inputs + ssd_scan_fwd_i8" if path == "w8a8" else "ssd_scan_fwd_bf16"}
 
     results = {}
     paths = (args.path,) if args.only_path else (args.path, "bf16" if args.path == "w8a8" else "w8a8")

@@ -2,7 +2,7 @@
 //   bf16 : H_0 = 0, H_{c+1} = exp(Acs_c[Q-1]) * H_c + S_c  (fp32; S_c stored as bf16)
 //   W8A8 : H_{c+1} = sat127(S8_c + ((dq_c * H_c + 2^(k-1)) >> k))       (int32, then INT8)
 // Every (p,n) element of a (b,h) state is an independent scalar recurrence, so one
-// thread owns 4 consecutive elements and walks the chunks; consecutive threads own
+// thread owns 4 (bf16 path) or 16 (W8A8) consecutive elements and walks the chunks; consecutive threads own
 // consecutive elements (coalesced vector loads and stores).  Loads of the next
 // kAhead chunks' S are issued ahead of the dependent updates.
 #include "kernels.h"
@@ -72,11 +72,13 @@ state_passing_bf16_kernel(Dims d, const TS* __restrict__ S, const float* __restr
     if (amax_h) atomic_max_nonneg(amax_h + h * d.P + e / d.N, amax);  // the 4 elements share p
 }
 
+constexpr int kVecI8 = 16;                               // INT8 elements per thread: one 16-byte load
+
 __global__ void __launch_bounds__(kThreads)
 state_passing_i8_kernel(Dims d, const int8_t* __restrict__ S8, const int32_t* __restrict__ dq,
                         int shift, int8_t* __restrict__ H8, int8_t* __restrict__ final_state) {
     const int PN = d.P * d.N;
-    const int e = (blockIdx.x * kThreads + threadIdx.x) * kVec;
+    const int e = (blockIdx.x * kThreads + threadIdx.x) * kVecI8;
     const int h = blockIdx.y, b = blockIdx.z;
     if (e >= PN) return;
     const long long stride = (long long)d.H * PN;
@@ -84,34 +86,42 @@ state_passing_i8_kernel(Dims d, const int8_t* __restrict__ S8, const int32_t* __
     int8_t* hc = H8 + ((long long)b * d.nc * d.H + h) * PN + e;
     const int32_t* q = dq + ((long long)b * d.H + h) * d.nc;
     const int half = 1 << (shift - 1);
-    int hv[kVec] = {0, 0, 0, 0};
-    auto pack = [](const int (&v)[kVec]) -> uint32_t {
-        return (uint32_t)(v[0] & 0xff) | ((uint32_t)(v[1] & 0xff) << 8) | ((uint32_t)(v[2] & 0xff) << 16) |
-               ((uint32_t)(v[3] & 0xff) << 24);
-    };
-    for (int c0 = 0; c0 < d.nc; c0 += kAhead) {
-        uint32_t sv[kAhead];
-        int qv[kAhead];
+    int hv[kVecI8];
 #pragma unroll
-        for (int i = 0; i < kAhead; ++i) {
+    for (int v = 0; v < kVecI8; ++v) hv[v] = 0;
+    auto pack = [&]() -> uint4 {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            w[i] = __byte_perm(__byte_perm(hv[4 * i], hv[4 * i + 1], 0x0040), __byte_perm(hv[4 * i + 2], hv[4 * i + 3], 0x0040),
+                               0x5410);
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    };
+    constexpr int kAheadI8 = 4;
+    for (int c0 = 0; c0 < d.nc; c0 += kAheadI8) {
+        uint4 sv[kAheadI8];
+        int qv[kAheadI8];
+#pragma unroll
+        for (int i = 0; i < kAheadI8; ++i) {
             const int c = c0 + i;
-            sv[i] = c < d.nc ? __ldg(reinterpret_cast<const unsigned int*>(s + c * stride)) : 0u;
+            sv[i] = c < d.nc ? __ldg(reinterpret_cast<const uint4*>(s + c * stride)) : make_uint4(0, 0, 0, 0);
             qv[i] = c < d.nc ? __ldg(q + c) : 0;
         }
 #pragma unroll
-        for (int i = 0; i < kAhead; ++i) {
+        for (int i = 0; i < kAheadI8; ++i) {
             const int c = c0 + i;
             if (c < d.nc) {
-                *reinterpret_cast<uint32_t*>(hc + c * stride) = pack(hv);
+                *reinterpret_cast<uint4*>(hc + c * stride) = pack();
+                const uint32_t w[4] = {sv[i].x, sv[i].y, sv[i].z, sv[i].w};
 #pragma unroll
-                for (int v = 0; v < kVec; ++v) {
-                    const int sc = (int)(int8_t)(sv[i] >> (8 * v));          // sign-extended code
+                for (int v = 0; v < kVecI8; ++v) {
+                    const int sc = (int)(int8_t)(w[v >> 2] >> (8 * (v & 3)));     // sign-extended code
                     hv[v] = sat127(sc + ((qv[i] * hv[v] + half) >> shift));
                 }
             }
         }
     }
-    *reinterpret_cast<uint32_t*>(final_state + ((long long)b * d.H + h) * PN + e) = pack(hv);
+    *reinterpret_cast<uint4*>(final_state + ((long long)b * d.H + h) * PN + e) = pack();
 }
 
 }  // namespace
@@ -134,8 +144,8 @@ cudaError_t launch_state_passing_bf16(const Dims& d, const void* S, bool s_fp32,
 cudaError_t launch_state_passing_i8(const Dims& d, const int8_t* S8, const int32_t* dq, int shift,
                                     int8_t* H8, int8_t* final_state, cudaStream_t st) {
     if (d.B == 0) return cudaSuccess;
-    if ((d.P * d.N) % kVec != 0) return cudaErrorInvalidValue;
-    dim3 grid((d.P * d.N / kVec + kThreads - 1) / kThreads, d.H, d.B);
+    if ((d.P * d.N) % kVecI8 != 0) return cudaErrorInvalidValue;
+    dim3 grid((d.P * d.N / kVecI8 + kThreads - 1) / kThreads, d.H, d.B);
     state_passing_i8_kernel<<<grid, kThreads, 0, st>>>(d, S8, dq, shift, H8, final_state);
     return cudaGetLastError();
 }

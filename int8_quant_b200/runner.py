@@ -111,3 +111,79 @@ class SsdProblem:
         ssd.ssd_scan_fwd_i8_debug(self.shape, i["x"], i["dt"], i["A"], self.Bq, self.Cq, i["D"], self.params,
                                   self.y, self.final8, self.ws_i8, dbg, stream)
         return dbg
+
+
+class StreamedScan:
+    """A batch held in pinned host memory, scanned in groups of batch rows with the copies
+    overlapped: group g's host->device copy, group g-1's scan and group g-2's device->host
+    copy run on three streams at once (batch rows are independent problems).
+
+    host: pinned CPU tensors x [B,L,H,P] (bf16), dt [B,L,H], B and C [B,L,G,N] (bf16), and
+    the outputs y [B,L,H,P] (bf16) and final [B,H,P,N] (fp32 for bf16, int8 for W8A8).
+    A and D live on the device.  W8A8 takes the static scales (device tensors).
+    """
+
+    def __init__(self, host: dict, A, D, chunk: int, path: str, rows_per_group: int = 1, scales=None,
+                 shift: int = 7, device="cuda"):
+        assert path in ("bf16", "w8a8")
+        self.h, self.path, self.A, self.D = host, path, A, D
+        b, L, H, P = host["x"].shape
+        G, N = host["B"].shape[2], host["B"].shape[3]
+        self.rows = rows_per_group
+        self.groups = [(r, min(rows_per_group, b - r)) for r in range(0, b, rows_per_group)]
+        self.shape = ssd.SsdShape.of(rows_per_group, L, H, P, G, N, chunk)
+        dev = torch.device(device)
+        i8 = path == "w8a8"
+        self.slots = []
+        for _ in range(2):
+            sl = {k: torch.empty((rows_per_group,) + tuple(host[k].shape[1:]), dtype=host[k].dtype, device=dev)
+                  for k in ("x", "dt", "B", "C", "y", "final")}
+            if i8:
+                sl["Bq"] = torch.empty(sl["B"].shape, dtype=torch.int8, device=dev)
+                sl["Cq"] = torch.empty(sl["C"].shape, dtype=torch.int8, device=dev)
+            self.slots.append(sl)
+        self.ws = torch.empty(max(ssd.ssd_workspace_bytes(self.shape, i8), 256), dtype=torch.uint8, device=dev)
+        if i8:
+            self.scales = scales
+            self.params = ssd.i8_params(scales["s_B"], scales["s_C"], scales["s_x"], scales["s_s"], shift)
+        self.streams = [torch.cuda.Stream(device=dev) for _ in range(3)]      # h2d, compute, d2h
+        self.ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "done", "out")}
+        self.seq = 0                                                           # groups enqueued so far
+        self.h2d_bytes = sum(host[k].numel() * host[k].element_size() for k in ("x", "dt", "B", "C"))
+        self.d2h_bytes = sum(host[k].numel() * host[k].element_size() for k in ("y", "final"))
+
+    def run(self):
+        """Enqueue the whole batch; returns at once (synchronise on `self.streams[2]`)."""
+        s_in, s_cmp, s_out = self.streams
+        for r0, n in self.groups:
+            g = self.seq
+            self.seq += 1
+            k = g % 2
+            sl = self.slots[k]
+            shape = self.shape if n == self.rows else ssd.SsdShape.of(
+                n, self.shape.seqlen, self.shape.nheads, self.shape.headdim, self.shape.ngroups, self.shape.dstate,
+                self.shape.chunk)
+            with torch.cuda.stream(s_in):
+                if g >= 2:
+                    s_in.wait_event(self.ev["done"][k])             # slot's inputs consumed by scan g-2
+                for name in ("x", "dt", "B", "C"):
+                    sl[name][:n].copy_(self.h[name][r0:r0 + n], non_blocking=True)
+                self.ev["in"][k].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(self.ev["in"][k])
+                if g >= 2:
+                    s_cmp.wait_event(self.ev["out"][k])            # slot's outputs read by copy g-2
+                if self.path == "w8a8":
+                    ssd.ssd_quantize_inputs(shape, sl["B"], sl["C"], self.scales["s_B"], self.scales["s_C"], sl["Bq"],
+                                            sl["Cq"], s_cmp)
+                    ssd.ssd_scan_fwd_i8(shape, sl["x"], sl["dt"], self.A, sl["Bq"], sl["Cq"], self.D, self.params,
+                                        sl["y"], sl["final"], self.ws, s_cmp)
+                else:
+                    ssd.ssd_scan_fwd_bf16(shape, sl["x"], sl["dt"], self.A, sl["B"], sl["C"], self.D, sl["y"],
+                                          sl["final"], self.ws, s_cmp)
+                self.ev["done"][k].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(self.ev["done"][k])
+                self.h["y"][r0:r0 + n].copy_(sl["y"][:n], non_blocking=True)
+                self.h["final"][r0:r0 + n].copy_(sl["final"][:n], non_blocking=True)
+                self.ev["out"][k].record(s_out)

@@ -145,3 +145,34 @@ def test_workspace_status_is_ok_after_a_run(torch_cuda):
     inp, pb = _problem(torch_cuda, CASES["tiny"])
     pb.run_bf16()
     assert iq.ssd_workspace_status(pb.ws_bf16) == 0
+
+
+@pytest.mark.parametrize("path", ["bf16", "w8a8"])
+@pytest.mark.parametrize("name", ["ragged-q256", "tiny-ragged"])
+def test_streamed_batch_equals_whole_batch(torch_cuda, name, path):
+    """Host-resident batch run group by group with overlapped copies (two rows per group,
+    so the last group is partial for an odd batch) gives the whole-batch results bit for bit."""
+    from int8_quant_b200.runner import StreamedScan
+    torch = torch_cuda
+    w = CASES[name].with_(batch=3)
+    inp, pb = _problem(torch_cuda, w)
+    if path == "w8a8":
+        sc = oracle_scales(inp, w.chunk, w.calib_prefix)
+        pb.set_scales(sc["s_B"], sc["s_C"], sc["s_x"], sc["s_s"], 7)
+        pb.run_i8()
+        fin = pb.final8
+    else:
+        pb.run_bf16()
+        fin = pb.final32
+    torch.cuda.synchronize()
+    host = {k: pb.inp[k].to("cpu").pin_memory() for k in ("x", "dt", "B", "C")}
+    host["y"] = torch.empty_like(pb.y, device="cpu").pin_memory()
+    host["final"] = torch.empty_like(fin, device="cpu").pin_memory()
+    run = StreamedScan(host, pb.inp["A"], pb.inp["D"], w.chunk, path, rows_per_group=2,
+                       scales=pb.scales if path == "w8a8" else None)
+    for _ in range(2):                      # a second pass reuses the slots behind the first
+        host["y"].zero_()
+        run.run()
+        torch.cuda.synchronize()
+        assert torch.equal(host["y"].view(torch.int16), pb.y.cpu().view(torch.int16))
+        assert torch.equal(host["final"], fin.cpu())
