@@ -76,7 +76,7 @@ struct Cfg {
     static constexpr int OFF_X = (OFF_B + B_BYTES + 1023) & ~1023;
     static constexpr int OFF_H = OFF_X + 2 * X_BYTES;
     static constexpr int OFF_VEC = OFF_H + NHB * H_BYTES;        // 2 slots x {acs, dtc, a2, vB, dtw}[Q]
-    static constexpr int VEC_SLOT = 5 * Q * 4;
+    static constexpr int VEC_SLOT = (kI8 ? 6 : 5) * Q * 4;
     static constexpr int OFF_BAR = OFF_VEC + 2 * VEC_SLOT;
     // barriers
     static constexpr int B_LOAD = 0, B_CB = 1, B_PACKED = 2, B_XFULL = 3, B_XEMPTY = 5, B_HFULL = 7,
@@ -134,6 +134,13 @@ __device__ __forceinline__ void sub_f32x2(float& r0, float& r1, float a0, float 
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// float(a) for |a| < 2^22, exactly, without a conversion instruction: 1.5 * 2^23 + a is
+// representable, so its bit pattern is 0x4B400000 + a.  The int32 accumulators here are
+// sums of at most 128 products of INT8 codes, |a| <= 128 * 127 * 127 < 2^22.
+__device__ __forceinline__ float small_int_to_float(uint32_t a) {
+    return __fsub_rn(__int_as_float((int)a + 0x4B400000), 12582912.0f);
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -189,7 +196,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
     auto vec = [&](int s, int which) -> float* {
         return reinterpret_cast<float*>(sm + K::OFF_VEC + s * K::VEC_SLOT + which * Q * 4);
     };
-    enum { kAcs = 0, kDtc = 1, kA2 = 2, kVB = 3, kDtw = 4 };
+    enum { kAcs = 0, kDtc = 1, kA2 = 2, kVB = 3, kDtw = 4, kMul = 5 };
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -393,8 +400,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float lo = kI8 ? (float)(int32_t)v[2 * i] : __uint_as_float(v[2 * i]);
-                        const float hi = kI8 ? (float)(int32_t)v[2 * i + 1] : __uint_as_float(v[2 * i + 1]);
+                        const float lo = kI8 ? small_int_to_float(v[2 * i]) : __uint_as_float(v[2 * i]);
+                        const float hi = kI8 ? small_int_to_float(v[2 * i + 1]) : __uint_as_float(v[2 * i + 1]);
                         w[i] = pack_bf16(lo, hi);
                     }
                     tc::tmem_st16(trow + (J == 0 ? K::CBP0 : K::CBP1) + g32 * 16, w);
@@ -534,6 +541,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 float* a2 = vec(s, kA2);
                 float* v32 = vec(s, kVB);
                 float* dtw = vec(s, kDtw);
+                if (kI8 && tid - kScaleWarp0 * 32 < kP) {
+                    // ChunkScan1's dequantisation s_C s_s[h,p] per column
+                    const int p = tid - kScaleWarp0 * 32;
+                    vec(s, kMul)[p] = __ldg(sc.s_C + g) * __ldg(sc.s_s + h * kP + p);
+                }
                 for (int i = tid - kScaleWarp0 * 32; i < Q; i += kEpiThreads) {
                     const float ai = acs[i] * kLog2e;
                     const float ar = acs[i | 31] * kLog2e;
@@ -567,7 +579,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         float f;
-                        if (kI8) f = (float)(int32_t)v[i] * (__ldg(sc.s_C + g) * __ldg(sc.s_s + h * kP + 32 * hf + i));
+                        if (kI8) f = small_int_to_float(v[i]) * vec(s, kMul)[32 * hf + i];
                         else f = __uint_as_float(v[i]);
                         v[i] = __float_as_uint(f * e);
                     }
