@@ -83,6 +83,12 @@ __device__ __forceinline__ void mul_f32x2(float& r0, float& r1, float a0, float 
         : "=f"(r0), "=f"(r1)
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
+__device__ __forceinline__ void sub_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
 // code_bits of two values, the rounding additions packed.
 __device__ __forceinline__ void code_bits2(int& q0, int& q1, float v0, float v1) {
     const float c0 = fminf(fmaxf(v0, -127.f), 127.f), c1 = fminf(fmaxf(v1, -127.f), 127.f);
@@ -305,15 +311,30 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                 for (int p = 0; p < kP; ++p)
                     S[base + p * kN] = float_to_bf16_bits(__uint_as_float(p < 32 ? v0[p] : v1[p - 32]));
             } else {
+                // |acc| <= Q * 127 * 127 < 2^22; the code's byte is the low byte of code_bits
 #pragma unroll
-                for (int p = 0; p < kP; ++p) {
-                    const int acc = (int)(p < 32 ? v0[p] : v1[p - 32]);
-                    const float mq = __shfl_sync(0xffffffffu, p < 32 ? c0 : c1, p & 31);
-                    // |acc| <= Q * 127 * 127 < 2^22
-                    const int q = code_bits(__fmul_rn(small_int_to_float(acc), mq)) - kRoundBits;
-                    S8[base + p * kN] = (int8_t)q;
-                    if (dbg.acc_state) dbg.acc_state[base + p * kN] = acc;
-                    if (dbg.S8) dbg.S8[base + p * kN] = (int8_t)q;
+                for (int p = 0; p < kP; p += 2) {
+                    const uint32_t a0 = p < 32 ? v0[p] : v1[p - 32], a1 = p < 32 ? v0[p + 1] : v1[p - 31];
+                    const float mq0 = __shfl_sync(0xffffffffu, p < 32 ? c0 : c1, p & 31);
+                    const float mq1 = __shfl_sync(0xffffffffu, p < 32 ? c0 : c1, (p + 1) & 31);
+                    float f0, f1, r0, r1;
+                    sub_f32x2(f0, f1, __int_as_float((int)a0 + kRoundBits), __int_as_float((int)a1 + kRoundBits), kRound,
+                              kRound);
+                    mul_f32x2(r0, r1, f0, f1, mq0, mq1);
+                    int q0, q1;
+                    code_bits2(q0, q1, r0, r1);
+                    S8[base + p * kN] = (int8_t)q0;
+                    S8[base + (p + 1) * kN] = (int8_t)q1;
+                }
+                if (dbg.acc_state || dbg.S8) {
+#pragma unroll
+                    for (int p = 0; p < kP; ++p) {
+                        const int acc = (int)(p < 32 ? v0[p] : v1[p - 32]);
+                        const float mq = __shfl_sync(0xffffffffu, p < 32 ? c0 : c1, p & 31);
+                        const int q = code_bits(__fmul_rn(small_int_to_float(acc), mq)) - kRoundBits;
+                        if (dbg.acc_state) dbg.acc_state[base + p * kN] = acc;
+                        if (dbg.S8) dbg.S8[base + p * kN] = (int8_t)q;
+                    }
                 }
             }
         }
