@@ -329,11 +329,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             const uint32_t u = (uint32_t)(it >> 1);
             if (yo == it && !(ok = issue_yo(true))) break;
             // waiting for this head's scaling: meanwhile start the next head's ChunkScan1
-            while (!ready(K::B_YSCALED + s, u & 1)) {
-                if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
-                if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-            }
-            if (!ok || !(ok = wait_all(K::B_YSCALED + s, u & 1))) break;
+            // one look at the next head's ChunkScan1, then a suspending wait (no spinning:
+            // the builders share this warp's scheduler)
+            if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
+            if (!(ok = wait_all(K::B_YSCALED + s, u & 1))) break;
             if (!(ok = wait_all(K::B_XFULL + s, u & 1))) break;
             const uint64_t dX = dX0 + (uint64_t)((s * K::X_BYTES) >> 4);
             const uint32_t ycol = tmem + K::YCOL + 128 * s;
@@ -342,11 +341,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 piece_of(Q, k, J, ib);
                 const int slot = p & (kRing - 1);
                 const uint32_t rpar = (uint32_t)((p / kRing) & 1);
-                while (!ready(K::B_RFULL + slot, rpar)) {
-                    if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
-                    if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-                }
-                if (!ok) break;
+                if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
+                if (!(ok = wait_all(K::B_RFULL + slot, rpar))) break;
                 tc::tc_fence_after();
                 if (tc::elect_one()) {
                     const uint32_t am = tmem + K::RING + slot * 32;      // 64 bf16 = 32 columns
