@@ -141,6 +141,13 @@ __device__ __forceinline__ float small_int_to_float(uint32_t a) {
     return __fsub_rn(__int_as_float((int)a + 0x4B400000), 12582912.0f);
 }
 
+// Two bf16 products (round to nearest even) in one packed instruction.
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -443,14 +450,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     const float4* v4 = reinterpret_cast<const float4*>(v32 + i0);
 #pragma unroll
                     for (int e4 = 0; e4 < 4; ++e4) {
+                        // the decay factors in fp32, rounded to bf16 pairs, times the CB pairs
                         const float4 f = v4[e4];
-                        float w0, w1, w2, w3, m0, m1, m2, m3;
+                        float w0, w1, w2, w3;
                         mul_f32x2(w0, w1, uj, uj, f.x, f.y);
                         mul_f32x2(w2, w3, uj, uj, f.z, f.w);
-                        mul_f32x2(m0, m1, bf16lo(v[2 * e4]), bf16hi(v[2 * e4]), w0, w1);
-                        mul_f32x2(m2, m3, bf16lo(v[2 * e4 + 1]), bf16hi(v[2 * e4 + 1]), w2, w3);
-                        out[2 * e4] = pack_bf16(m0, m1);
-                        out[2 * e4 + 1] = pack_bf16(m2, m3);
+                        out[2 * e4] = mul_bf16x2(v[2 * e4], pack_bf16(w0, w1));
+                        out[2 * e4 + 1] = mul_bf16x2(v[2 * e4 + 1], pack_bf16(w2, w3));
                     }
                 } else if (jb == cb) {
                     // masked entries (column > row) have a positive exponent; they are
@@ -463,14 +469,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                         float x0, x1, x2, x3;
                         sub_f32x2(x0, x1, aj, aj, av.x, av.y);
                         sub_f32x2(x2, x3, aj, aj, av.z, av.w);
-                        float t0, t1, t2, t3, m0, m1, m2, m3;
+                        float t0, t1, t2, t3;
                         mul_f32x2(t0, t1, ex2(x0), ex2(x1), dv.x, dv.y);
                         mul_f32x2(t2, t3, ex2(x2), ex2(x3), dv.z, dv.w);
-                        mul_f32x2(m0, m1, bf16lo(v[2 * e4]), bf16hi(v[2 * e4]), t0, t1);
-                        mul_f32x2(m2, m3, bf16lo(v[2 * e4 + 1]), bf16hi(v[2 * e4 + 1]), t2, t3);
                         const int c = c0 + 4 * e4;                // column within the block; the row is `lane`
-                        out[2 * e4] = pack_bf16(c <= lane ? m0 : 0.f, c + 1 <= lane ? m1 : 0.f);
-                        out[2 * e4 + 1] = pack_bf16(c + 2 <= lane ? m2 : 0.f, c + 3 <= lane ? m3 : 0.f);
+                        out[2 * e4] = mul_bf16x2(v[2 * e4], pack_bf16(c <= lane ? t0 : 0.f, c + 1 <= lane ? t1 : 0.f));
+                        out[2 * e4 + 1] =
+                            mul_bf16x2(v[2 * e4 + 1], pack_bf16(c + 2 <= lane ? t2 : 0.f, c + 3 <= lane ? t3 : 0.f));
                     }
                 } else {
 #pragma unroll
