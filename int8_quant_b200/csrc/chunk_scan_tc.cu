@@ -127,6 +127,17 @@ __device__ __forceinline__ void mul_f32x2(float& r0, float& r1, float a0, float 
         : "=f"(r0), "=f"(r1)
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
+__device__ __forceinline__ void add_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ void sub_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
     asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
         "sub.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
@@ -427,6 +438,14 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         // one exponential per element; above it is zero.  The next piece's CB columns
         // are loaded from TMEM while the current piece is computed.
         const int c0 = 16 * set;                                  // first column within a block
+        // diagonal blocks: which halves of this row's column pairs (c0 + 2k, c0 + 2k + 1)
+        // lie on or below the diagonal (column <= row = lane)
+        uint32_t dmask[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int c = c0 + 2 * k;
+            dmask[k] = c + 1 <= lane ? 0xffffffffu : (c == lane ? 0x0000ffffu : 0u);
+        }
         int p = 0;
         for (int it = 0; ok && it < nh; ++it) {
             const int s = it & 1;
@@ -446,36 +465,31 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             auto build16 = [&](const uint32_t (&v)[8], int jb, int cb, float aj, uint32_t (&out)[8]) {
                 const int i0 = 32 * cb + c0;
                 if (jb > cb) {
+                    // row factor and column factors as bf16 pairs: two bf16x2 products per pair
                     const float uj = ex2(fminf(aj - a2[32 * cb + 31], 0.f));
-                    const float4* v4 = reinterpret_cast<const float4*>(v32 + i0);
+                    const uint32_t ub = pack_bf16(uj, uj);
+                    const uint4* v4 = reinterpret_cast<const uint4*>(reinterpret_cast<const uint32_t*>(v32) + i0 / 2);
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        // the decay factors in fp32, rounded to bf16 pairs, times the CB pairs
-                        const float4 f = v4[e4];
-                        float w0, w1, w2, w3;
-                        mul_f32x2(w0, w1, uj, uj, f.x, f.y);
-                        mul_f32x2(w2, w3, uj, uj, f.z, f.w);
-                        out[2 * e4] = mul_bf16x2(v[2 * e4], pack_bf16(w0, w1));
-                        out[2 * e4 + 1] = mul_bf16x2(v[2 * e4 + 1], pack_bf16(w2, w3));
+                    for (int q = 0; q < 2; ++q) {
+                        const uint4 f = v4[q];
+                        out[4 * q] = mul_bf16x2(v[4 * q], mul_bf16x2(ub, f.x));
+                        out[4 * q + 1] = mul_bf16x2(v[4 * q + 1], mul_bf16x2(ub, f.y));
+                        out[4 * q + 2] = mul_bf16x2(v[4 * q + 2], mul_bf16x2(ub, f.z));
+                        out[4 * q + 3] = mul_bf16x2(v[4 * q + 3], mul_bf16x2(ub, f.w));
                     }
                 } else if (jb == cb) {
-                    // masked entries (column > row) have a positive exponent; they are
-                    // selected away, whatever the exponential gives
-                    const float4* a4 = reinterpret_cast<const float4*>(a2 + i0);
-                    const float4* d4 = reinterpret_cast<const float4*>(dtw + i0);
+                    // exp(Acs_j - Acs_i) dt_i = 2^(a_j + (log2(dt_i) - a_i)), the column term
+                    // prepared per head; masked entries (column > row) may overflow to inf
+                    // and are cleared bitwise by the row's pair masks
+                    const float4* l4 = reinterpret_cast<const float4*>(dtw + i0);
 #pragma unroll
                     for (int e4 = 0; e4 < 4; ++e4) {
-                        const float4 av = a4[e4], dv = d4[e4];
+                        const float4 lv = l4[e4];
                         float x0, x1, x2, x3;
-                        sub_f32x2(x0, x1, aj, aj, av.x, av.y);
-                        sub_f32x2(x2, x3, aj, aj, av.z, av.w);
-                        float t0, t1, t2, t3;
-                        mul_f32x2(t0, t1, ex2(x0), ex2(x1), dv.x, dv.y);
-                        mul_f32x2(t2, t3, ex2(x2), ex2(x3), dv.z, dv.w);
-                        const int c = c0 + 4 * e4;                // column within the block; the row is `lane`
-                        out[2 * e4] = mul_bf16x2(v[2 * e4], pack_bf16(c <= lane ? t0 : 0.f, c + 1 <= lane ? t1 : 0.f));
-                        out[2 * e4 + 1] =
-                            mul_bf16x2(v[2 * e4 + 1], pack_bf16(c + 2 <= lane ? t2 : 0.f, c + 3 <= lane ? t3 : 0.f));
+                        add_f32x2(x0, x1, aj, aj, lv.x, lv.y);
+                        add_f32x2(x2, x3, aj, aj, lv.z, lv.w);
+                        out[2 * e4] = mul_bf16x2(v[2 * e4], pack_bf16(ex2(x0), ex2(x1))) & dmask[2 * e4];
+                        out[2 * e4 + 1] = mul_bf16x2(v[2 * e4 + 1], pack_bf16(ex2(x2), ex2(x3))) & dmask[2 * e4 + 1];
                     }
                 } else {
 #pragma unroll
@@ -552,8 +566,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     const float ar = acs[i | 31] * kLog2e;
                     const float dw = dts[i] * sCB;
                     a2[i] = ai;
-                    dtw[i] = dw;
-                    v32[i] = ex2(fminf(ar - ai, 0.f)) * dw;
+                    dtw[i] = lg2(dw) - ai;                        // log2(dt_i) - a_i; -inf when dt_i = 0
+                    // column factors as bf16 pairs (consecutive lanes hold consecutive i)
+                    const float vi = ex2(fminf(ar - ai, 0.f)) * dw;
+                    const float vn = __shfl_down_sync(0xffffffffu, vi, 1);
+                    if ((i & 1) == 0) reinterpret_cast<uint32_t*>(v32)[i / 2] = pack_bf16(vi, vn);
                 }
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar + K::B_VPREP + s);
