@@ -120,13 +120,7 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Two IEEE fp32 operations (round to nearest even) in one packed instruction.
-__device__ __forceinline__ void mul_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
-    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "mul.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
-        : "=f"(r0), "=f"(r1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
+// Two IEEE fp32 additions (round to nearest even) in one packed instruction.
 __device__ __forceinline__ void add_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
     asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
         "add.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
@@ -137,12 +131,6 @@ __device__ __forceinline__ float lg2(float x) {
     float y;
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-__device__ __forceinline__ void sub_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
-    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "sub.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
-        : "=f"(r0), "=f"(r1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
 // float(a) for |a| < 2^22, exactly, without a conversion instruction: 1.5 * 2^23 + a is
