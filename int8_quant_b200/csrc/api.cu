@@ -43,8 +43,41 @@ ssd_status make_dims(const ssd_shape* s, Dims* d) {
 // CUDA-core kernels.
 bool tensor_core_shape(const Dims& d) { return d.P == 64 && d.N == 128; }
 
-// Heads that share one ChunkBMM result in the tensor-core ChunkScan.
-constexpr int kHeadsPerScanCta = 8;
+}  // namespace
+
+int device_sm_count() {
+    static int n[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (n[dev] == 0) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        n[dev] = v > 0 ? v : 1;
+    }
+    return n[dev];
+}
+
+namespace {
+
+// Heads that share one ChunkBMM result in a tensor-core ChunkScan CTA.  One CTA runs per
+// SM, so the grid runs in waves; a CTA costs about one head's time for its prologue (C and
+// B tiles, ChunkBMM, packing) plus one per head.  Among a few block sizes, take the one
+// whose waves x (1 + heads) is smallest: fewer prologues against a full last wave.
+int scan_heads_per_cta(const Dims& d) {
+    const int sms = device_sm_count();
+    int best = 8;
+    long long best_cost = -1;
+    for (int hpc : {8, 10, 12, 16, 20}) {
+        const int per = hpc < d.hpg ? hpc : d.hpg;
+        const long long ctas = (long long)d.G * ((d.hpg + per - 1) / per) * d.nc * d.B;
+        const long long cost = ((ctas + sms - 1) / sms) * (1 + per);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = per;
+        }
+    }
+    return best;
+}
 
 // The CUDA error behind this thread's last SSD_ERR_CUDA (cudaSuccess if none).
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
@@ -232,7 +265,7 @@ ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const fl
     SSD_STAGE("state_passing", launch_state_passing_bf16(d, S, !tcs, decay, Hc, final_state, nullptr, stream));
     if (tensor_core_shape(d))
         SSD_STAGE("chunk_scan", launch_chunk_scan_tc(d, false, x, B, C, Acs, dtc, D, I8Scales{}, Hc, y, nullptr,
-                                                     kHeadsPerScanCta, status, stream));
+                                                     scan_heads_per_cta(d), status, stream));
     else
         SSD_STAGE("chunk_scan", launch_chunk_scan_bf16(d, x, dt, Acs, B, C, D, Hc, y, stream));
     return SSD_OK;
@@ -278,7 +311,7 @@ ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, cons
     SSD_STAGE("state_passing", launch_state_passing_i8(d, S8, dq, sc.shift, H8, final_state, stream));
     if (tensor_core_shape(d))
         SSD_STAGE("chunk_scan", launch_chunk_scan_tc(d, true, x, Bq, Cq, Acs, dtc, D, sc, H8, y, dbg ? &dd : nullptr,
-                                                     kHeadsPerScanCta, status, stream));
+                                                     scan_heads_per_cta(d), status, stream));
     else
         SSD_STAGE("chunk_scan", launch_chunk_scan_i8(d, x, dt, Acs, Bq, Cq, D, sc, H8, y, dbg ? &dd : nullptr, stream));
     if (dbg) {

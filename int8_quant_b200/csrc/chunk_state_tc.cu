@@ -421,19 +421,6 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     if (warp == 1) tc::tmem_dealloc(tmem, kAcc * 64);
 }
 
-int sm_count() {
-    static int n[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (n[dev] == 0) {
-        int v = 0;
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-        n[dev] = v > 0 ? v : 1;
-    }
-    return n[dev];
-}
-
 template <int Q, bool kI8>
 cudaError_t launch_q(const Dims& d, const CUtensorMap& tx, const CUtensorMap& tb, const float* lut,
                      const float* inv_sx, const float* mq, uint16_t* S, int8_t* S8, const I8Debug* dbg, int* status,
@@ -444,7 +431,8 @@ cudaError_t launch_q(const Dims& d, const CUtensorMap& tx, const CUtensorMap& tb
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const long long units = (long long)d.B * d.nc * d.H;
-    const int grid = (int)(units < sm_count() ? units : sm_count());
+    const int sms = device_sm_count();
+    const int grid = (int)(units < sms ? units : sms);
     I8Debug none{};
     k<<<grid, kThreads, smem, st>>>(tx, tb, d, lut, inv_sx, mq, S, S8, dbg ? *dbg : none, status);
     return cudaGetLastError();

@@ -107,6 +107,9 @@ cudaError_t launch_chunk_state_tc(const Dims& d, bool i8, const uint16_t* x, con
                                   const float* lut, const float* inv_sx, const float* mq, uint16_t* S, int8_t* S8,
                                   const I8Debug* dbg, int* status, cudaStream_t st);
 
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
+
 // Calibration helpers.
 cudaError_t launch_amax_bc(const Dims& d, const uint16_t* B, const uint16_t* C, float* amax_B,
                            float* amax_C, cudaStream_t st);
