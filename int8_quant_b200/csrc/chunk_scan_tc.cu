@@ -347,7 +347,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 piece_of(Q, k, J, ib);
                 const int slot = p & (kRing - 1);
                 const uint32_t rpar = (uint32_t)((p / kRing) & 1);
-                if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
+                // W8A8: the next head's (cheaper, int8) ChunkScan1 may go between the pieces
+                if (kI8 && yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
                 if (!(ok = wait_all(K::B_RFULL + slot, rpar))) break;
                 tc::tc_fence_after();
                 if (tc::elect_one()) {
@@ -362,6 +363,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             }
             if (!ok) break;
             if (tc::elect_one()) tc::mma_commit(bar + K::B_YFULL + s);
+            // bf16: the next head's ChunkScan1 goes behind this head's pieces in the tensor pipe
+            if (!kI8 && yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
             __syncwarp();
         }
     } else if (warp < kScaleWarp0) {
