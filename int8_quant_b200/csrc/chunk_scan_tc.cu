@@ -127,6 +127,20 @@ __device__ __forceinline__ void add_f32x2(float& r0, float& r1, float a0, float 
         : "=f"(r0), "=f"(r1)
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
+__device__ __forceinline__ void mul_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// r = a * b + c on fp32 pairs, fused, round to nearest even
+__device__ __forceinline__ void fma_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1, float c0,
+                                          float c1) {
+    asm("{\n\t.reg .b64 a, b, c, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mov.b64 c, {%6, %7};\n\tfma.rn.f32x2 r, a, b, c;\n\tmov.b64 {%0, %1}, r;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
 __device__ __forceinline__ float lg2(float x) {
     float y;
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -586,11 +600,20 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                         for (int i = 0; i < 32; ++i) dst[i] = (int32_t)v[i];
                     }
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        float f;
-                        if (kI8) f = small_int_to_float(v[i]) * vec(s, kMul)[32 * hf + i];
-                        else f = __uint_as_float(v[i]);
-                        v[i] = __float_as_uint(f * e);
+                    for (int i = 0; i < 32; i += 2) {
+                        float f0, f1;
+                        if (kI8) {
+                            const float2 m = *reinterpret_cast<const float2*>(vec(s, kMul) + 32 * hf + i);
+                            add_f32x2(f0, f1, __int_as_float((int)v[i] + 0x4B400000),
+                                      __int_as_float((int)v[i + 1] + 0x4B400000), -12582912.0f, -12582912.0f);
+                            mul_f32x2(f0, f1, f0, f1, m.x, m.y);
+                        } else {
+                            f0 = __uint_as_float(v[i]);
+                            f1 = __uint_as_float(v[i + 1]);
+                        }
+                        mul_f32x2(f0, f1, f0, f1, e, e);
+                        v[i] = __float_as_uint(f0);
+                        v[i + 1] = __float_as_uint(f1);
                     }
                     tc::tmem_st32(ybase + 64 * J + 32 * hf, v);
                 }
@@ -635,9 +658,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                             const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
                             uint32_t o[4];
 #pragma unroll
-                            for (int e2 = 0; e2 < 4; ++e2)
-                                o[e2] = pack_bf16(__uint_as_float(v[q * 8 + 2 * e2]) + Dh * bf16lo(xw[e2]),
-                                                  __uint_as_float(v[q * 8 + 2 * e2 + 1]) + Dh * bf16hi(xw[e2]));
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                float o0, o1;
+                                fma_f32x2(o0, o1, Dh, Dh, bf16lo(xw[e2]), bf16hi(xw[e2]), __uint_as_float(v[q * 8 + 2 * e2]),
+                                          __uint_as_float(v[q * 8 + 2 * e2 + 1]));
+                                o[e2] = pack_bf16(o0, o1);
+                            }
                             *px = make_uint4(o[0], o[1], o[2], o[3]);
                         }
                     }
