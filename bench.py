@@ -87,10 +87,10 @@ def measured_peaks():
 NCU_TRAFFIC = {
     # batch-2 capture scaled x4 to the batch-8 launch (traffic grows with the batch);
     # see profiles/chunk_scan_tc_mamba2-2.7b-b2.md
-    ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.653312e6 + 129.440512e6),
-                                            "src_sha1": "37e9f4c1cc4b22536816c1e3d85d4e6bd2f95fcc"},
-    ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (270.715648e6 + 130.753280e6),
-                                            "src_sha1": "37e9f4c1cc4b22536816c1e3d85d4e6bd2f95fcc"},
+    ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.526592e6 + 128.723200e6),
+                                            "src_sha1": "b837bf44032720a502f416f234d9dcca352800c3"},
+    ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (270.617856e6 + 132.557056e6),
+                                            "src_sha1": "b837bf44032720a502f416f234d9dcca352800c3"},
 }
 
 
