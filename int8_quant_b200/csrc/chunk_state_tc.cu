@@ -83,12 +83,6 @@ __device__ __forceinline__ void mul_f32x2(float& r0, float& r1, float a0, float 
         : "=f"(r0), "=f"(r1)
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
-__device__ __forceinline__ void sub_f32x2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
-    asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "sub.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
-        : "=f"(r0), "=f"(r1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
 // code_bits of two values, the rounding additions packed.
 __device__ __forceinline__ void code_bits2(int& q0, int& q1, float v0, float v1) {
     const float c0 = fminf(fmaxf(v0, -127.f), 127.f), c1 = fminf(fmaxf(v1, -127.f), 127.f);
@@ -318,8 +312,9 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                     const float mq0 = __shfl_sync(0xffffffffu, p < 32 ? c0 : c1, p & 31);
                     const float mq1 = __shfl_sync(0xffffffffu, p < 32 ? c0 : c1, (p + 1) & 31);
                     float f0, f1, r0, r1;
-                    sub_f32x2(f0, f1, __int_as_float((int)a0 + kRoundBits), __int_as_float((int)a1 + kRoundBits), kRound,
-                              kRound);
+                    // int-to-float conversions: they run on a pipe of their own, which is idle here
+                    f0 = __int2float_rn((int)a0);
+                    f1 = __int2float_rn((int)a1);
                     mul_f32x2(r0, r1, f0, f1, mq0, mq1);
                     int q0, q1;
                     code_bits2(q0, q1, r0, r1);
