@@ -53,13 +53,22 @@ cumsum_kernel(Dims d, const float* __restrict__ dt, const float* __restrict__ A,
     float* tile = smem;                             // [kHeadsPerCta][ld]  dt
     float* part = smem + kHeadsPerCta * ld;         // [kHeadsPerCta][ld]  Acs
     const int c = blockIdx.x, h0 = blockIdx.y * kHeadsPerCta, b = blockIdx.z;
-    for (int idx = threadIdx.x; idx < Q * kHeadsPerCta; idx += kThreads) {
+    // all of this thread's loads first (Q * 8 / 256 <= 8), then the shared-memory stores
+    constexpr int kLoads = 256 * kHeadsPerCta / kThreads;      // enough for Q = 256
+    float vals[kLoads];
+#pragma unroll
+    for (int r = 0; r < kLoads; ++r) {
+        const int idx = threadIdx.x + r * kThreads;
         const int j = idx / kHeadsPerCta, k = idx % kHeadsPerCta;
         const long long t = (long long)c * Q + j;
         const int h = h0 + k;
-        float v = 0.f;
-        if (t < d.L && h < d.H) v = __ldg(dt + ((long long)b * d.Ls + t) * d.H + h);
-        tile[k * ld + pad(j)] = v;
+        vals[r] = (j < Q && t < d.L && h < d.H) ? __ldg(dt + ((long long)b * d.Ls + t) * d.H + h) : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < kLoads; ++r) {
+        const int idx = threadIdx.x + r * kThreads;
+        const int j = idx / kHeadsPerCta, k = idx % kHeadsPerCta;
+        if (j < Q) tile[k * ld + pad(j)] = vals[r];
     }
     __syncthreads();
     const int k = threadIdx.x >> 5, lane = threadIdx.x & 31;

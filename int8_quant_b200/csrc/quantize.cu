@@ -17,20 +17,32 @@ quantize_bc_kernel(const uint4* __restrict__ B, const uint4* __restrict__ C,
     uint2* dst = blockIdx.y == 0 ? Bq : Cq;
     const float* s = blockIdx.y == 0 ? s_B : s_C;
     const int vec_per_group = N / 8;
-    for (long long i = blockIdx.x * (long long)kThreads + threadIdx.x; i < nvec;
-         i += (long long)gridDim.x * kThreads) {
-        const int g = (int)((i / vec_per_group) % G);
-        const float inv = __frcp_rn(__ldg(s + g));     // IEEE 1/s
-        const uint4 v = __ldg(src + i);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t out[2] = {0u, 0u};
+    const long long stride = (long long)gridDim.x * kThreads;
+    constexpr int kUnroll = 4;                           // loads in flight per thread
+    for (long long i0 = blockIdx.x * (long long)kThreads + threadIdx.x; i0 < nvec; i0 += kUnroll * stride) {
+        uint4 vv[kUnroll];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const uint16_t bits = (uint16_t)(w[k >> 1] >> ((k & 1) * 16));
-            const int q = quant_i8(bf16_bits_to_float(bits), inv);
-            out[k >> 2] |= ((uint32_t)(q & 0xff)) << ((k & 3) * 8);
+        for (int r = 0; r < kUnroll; ++r) {
+            const long long i = i0 + r * stride;
+            vv[r] = i < nvec ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
         }
-        dst[i] = make_uint2(out[0], out[1]);
+#pragma unroll
+        for (int r = 0; r < kUnroll; ++r) {
+            const long long i = i0 + r * stride;
+            if (i >= nvec) break;
+            const int g = (int)((i / vec_per_group) % G);
+            const float inv = __frcp_rn(__ldg(s + g));     // IEEE 1/s
+            const uint4 v = vv[r];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t out[2] = {0u, 0u};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint16_t bits = (uint16_t)(w[k >> 1] >> ((k & 1) * 16));
+                const int q = quant_i8(bf16_bits_to_float(bits), inv);
+                out[k >> 2] |= ((uint32_t)(q & 0xff)) << ((k & 3) * 8);
+            }
+            dst[i] = make_uint2(out[0], out[1]);
+        }
     }
 }
 
