@@ -112,27 +112,70 @@ def traffic_for(kernel: str, path: str, workload: str):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event (throttle) reasons of the GPU, read through NVML every
+    millisecond on a background thread while the context is open (read-only queries;
+    the timed steps last milliseconds, below nvidia-smi's sampling interval).  Falls
+    back to an nvidia-smi subprocess when NVML is not importable."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+    SMI_Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"ssd_bench_clocks_{os.getpid()}.csv")
+    def __init__(self, device):
+        self.device = device
+        self.samples = []            # (sm MHz, max sm MHz, set of reasons)
+        self.source = None
+        self.err = None
+
+    def _uuid(self):
+        try:
+            u = str(torch.cuda.get_device_properties(self.device).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            return None
+
+    def _nvml_loop(self, nv, h):
+        names = [(n, getattr(nv, c)) for n, c in self.REASONS if hasattr(nv, c)]
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.samples.append((float(sm), float(mx), {n for n, b in names if bits & b}))
+            self._stop.wait(0.001)
 
     def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        self._thread = self.proc = None
         try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.fh,
-                                         stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            uuid = self._uuid()
+            h = nv.nvmlDeviceGetHandleByUUID(uuid) if uuid else nv.nvmlDeviceGetHandleByIndex(self.device.index)
+            self._thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self._thread.start()
+            self.source = "nvml, 1 ms"
+        except Exception as e:                 # no NVML: nvidia-smi at its fastest interval
+            self.err = f"nvml: {e}"
+            try:
+                self.path = os.path.join("/tmp", f"ssd_bench_clocks_{os.getpid()}.csv")
+                self.fh = open(self.path, "w")
+                gpu = self._uuid() or str(self.device.index)
+                self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.SMI_Q}", "--format=csv,noheader,nounits",
+                                              "-i", gpu, "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+                self.source = "nvidia-smi, 100 ms"
+            except (OSError, FileNotFoundError):
+                self.proc = None
         return self
 
     def __exit__(self, *a):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
         if self.proc:
             self.proc.terminate()
             try:
@@ -140,31 +183,29 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
             self.fh.close()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    try:
+                        self.samples.append((float(parts[1]), float(parts[2]),
+                                             {n for n, v in zip(names, parts[5:9]) if v.lower() == "active"}))
+                    except (ValueError, IndexError):
+                        continue
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
 
     def summary(self):
-        if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
-        try:
-            os.remove(self.path)
-        except OSError:
-            pass
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.source:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": f"unavailable ({self.err})"}
+        sm = [x[0] for x in self.samples]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(x[1] for x in self.samples) if sm else None,
+                "reasons": sorted(set().union(*[x[2] for x in self.samples])) if sm else [],
+                "samples": len(sm), "source": self.source}
 
 
 # ---------------------------------------------------------------- CPU oracle baseline
@@ -275,7 +316,7 @@ def run_ours(args, rank, world, dist):
         torch.cuda.synchronize()
         iq.ssd_profile_reset()
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with ClockSampler(dev.index) as clk:
+        with ClockSampler(dev) as clk:
             barrier()
             torch.cuda.synchronize()
             iq.ssd_profile_enable(True)

@@ -98,7 +98,11 @@ __device__ __forceinline__ void piece_of(int Q, int k, int& J, int& ib) {
     }
 }
 
-// Bounded mbarrier wait that gives up early once another role has aborted.
+// Bounded mbarrier wait that gives up early once another role has aborted.  With
+// kBackoff a failed poll sleeps 20 ns before the next: in the W8A8 instantiation the
+// polls of waiting roles slowed the others measurably (a few per cent of the kernel);
+// in the bf16 one the sleep cost more than it saved.
+template <bool kBackoff = false>
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
     const long long t0 = clock64();
     while (!tc::mbar_try_wait(bar, parity)) {
@@ -108,6 +112,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
             if (status) atomicExch(status, kStatusTimeout);
             return false;
         }
+        if (kBackoff) __nanosleep(20);
     }
     return true;
 }
@@ -239,20 +244,20 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             for (int it = 0; it < nh; ++it) {
                 const int h = h0 + it, s = it & 1;
                 const uint32_t u = (uint32_t)(it >> 1);
-                if (!wait_bar(bar + K::B_VEMPTY + s, (u & 1) ^ 1, abort_flag, status)) break;
+                if (!wait_bar<kI8>(bar + K::B_VEMPTY + s, (u & 1) ^ 1, abort_flag, status)) break;
                 tc::mbar_arrive_expect_tx(bar + K::B_VFULL + s, 2 * Q * 4);
                 const long long vr = vec_row0 + (long long)h * d.nc * Q;
                 tc::bulk_load(vec(s, kAcs), Acs + vr, Q * 4, bar + K::B_VFULL + s);
                 tc::bulk_load(vec(s, kDtc), dtc + vr, Q * 4, bar + K::B_VFULL + s);
                 const int hb = kI8 ? s : 0;
                 const uint32_t hpar = kI8 ? ((u & 1) ^ 1) : (((uint32_t)it & 1) ^ 1);
-                if (!wait_bar(bar + K::B_HEMPTY + hb, hpar, abort_flag, status)) break;
+                if (!wait_bar<kI8>(bar + K::B_HEMPTY + hb, hpar, abort_flag, status)) break;
                 tc::mbar_arrive_expect_tx(bar + K::B_HFULL + hb, K::H_BYTES);
                 const int hrow = (int)((hc_row0 + h) * kP);
                 uint8_t* hdst = sm + K::OFF_H + hb * K::H_BYTES;
                 tc::tma_load_2d(hdst, &tm_h, bar + K::B_HFULL + hb, 0, hrow);
                 if (!kI8) tc::tma_load_2d(hdst + kP * 128, &tm_h, bar + K::B_HFULL + hb, 64, hrow);
-                if (!wait_bar(bar + K::B_XEMPTY + s, (u & 1) ^ 1, abort_flag, status)) break;
+                if (!wait_bar<kI8>(bar + K::B_XEMPTY + s, (u & 1) ^ 1, abort_flag, status)) break;
                 tc::mbar_arrive_expect_tx(bar + K::B_XFULL + s, K::X_BYTES);
                 tc::tma_load_3d(sm + K::OFF_X + s * K::X_BYTES, &tm_x, bar + K::B_XFULL + s, h * kP, c * Q, b);
             }
@@ -274,7 +279,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             return kI8 ? (uint32_t)(s * 32) : (uint32_t)((s >> 2) * rows * 128 + (s & 3) * 32);
         };
         auto wait_all = [&](int which, uint32_t parity) -> bool {
-            return __all_sync(0xffffffffu, wait_bar(bar + which, parity, abort_flag, status));
+            return __all_sync(0xffffffffu, wait_bar<kI8>(bar + which, parity, abort_flag, status));
         };
         auto ready = [&](int which, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, tc::mbar_test(bar + which, parity));
@@ -387,7 +392,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         const int quarter = warp & 3;
         const int rrow = quarter * 32 + lane;                 // row within a 128-row tile
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-        bool ok = tc::named_and(kIdBuild, kBuilderThreads, wait_bar(bar + K::B_CB, 0, abort_flag, status));
+        bool ok = tc::named_and(kIdBuild, kBuilderThreads, wait_bar<kI8>(bar + K::B_CB, 0, abort_flag, status));
         tc::tc_fence_after();
         if (ok && set == 0) {
             if (kI8 && dbg.cb && (blockIdx.x % ctas_per_group) == 0) {
@@ -431,7 +436,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar + K::B_PACKED);
         }
-        ok = tc::named_and(kIdBuild, kBuilderThreads, ok && wait_bar(bar + K::B_PACKED, 0, abort_flag, status));
+        ok = tc::named_and(kIdBuild, kBuilderThreads, ok && wait_bar<kI8>(bar + K::B_PACKED, 0, abort_flag, status));
         tc::tc_fence_after();
         // Every piece is built by all eight warps.  Warp (set, quarter) owns the 32
         // rows of its TMEM lane quarter and, of the piece's four 16-column groups, the
@@ -456,7 +461,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             const int s = it & 1;
             const uint32_t u = (uint32_t)(it >> 1);
             // the scalers have prepared the head's decay vectors
-            ok = __all_sync(0xffffffffu, wait_bar(bar + K::B_VPREP + s, u & 1, abort_flag, status));
+            ok = __all_sync(0xffffffffu, wait_bar<kI8>(bar + K::B_VPREP + s, u & 1, abort_flag, status));
             if (!ok) break;
             const float* a2 = vec(s, kA2);
             const float* v32 = vec(s, kVB);
@@ -521,7 +526,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 uint32_t out0[8], out1[8];
                 build16(cbv[k & 1][0], jb, 2 * ib, aj, out0);
                 build16(cbv[k & 1][1], jb, 2 * ib + 1, aj, out1);
-                if (!__all_sync(0xffffffffu, wait_bar(bar + K::B_REMPTY + slot, (uint32_t)(((pp / kRing) & 1) ^ 1),
+                if (!__all_sync(0xffffffffu, wait_bar<kI8>(bar + K::B_REMPTY + slot, (uint32_t)(((pp / kRing) & 1) ^ 1),
                                                       abort_flag, status))) {
                     ok = false;
                     break;
@@ -550,7 +555,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         for (int it = 0; ok && it < nh; ++it) {
             const int h = h0 + it, s = it & 1;
             const uint32_t u = (uint32_t)(it >> 1);
-            if (!(ok = tc::named_and(kIdScale, kEpiThreads, wait_bar(bar + K::B_VFULL + s, u & 1, abort_flag, status))))
+            if (!(ok = tc::named_and(kIdScale, kEpiThreads, wait_bar<kI8>(bar + K::B_VFULL + s, u & 1, abort_flag, status))))
                 break;
             {
                 // the builders' decay vectors: log2-scaled Acs, dt with CB's
@@ -580,7 +585,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar + K::B_VPREP + s);
             }
-            if (!(ok = tc::named_and(kIdScale, kEpiThreads, wait_bar(bar + K::B_YOFULL + s, u & 1, abort_flag, status))))
+            if (!(ok = tc::named_and(kIdScale, kEpiThreads, wait_bar<kI8>(bar + K::B_YOFULL + s, u & 1, abort_flag, status))))
                 break;
             tc::tc_fence_after();
             const float* acs = vec(s, kAcs);
@@ -635,8 +640,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         for (int it = 0; ok && it < nh; ++it) {
             const int h = h0 + it, s = it & 1;
             const uint32_t u = (uint32_t)(it >> 1);
-            bool w = wait_bar(bar + K::B_YFULL + s, u & 1, abort_flag, status);
-            w = w && wait_bar(bar + K::B_XFULL + s, u & 1, abort_flag, status);
+            bool w = wait_bar<kI8>(bar + K::B_YFULL + s, u & 1, abort_flag, status);
+            w = w && wait_bar<kI8>(bar + K::B_XFULL + s, u & 1, abort_flag, status);
             if (!(ok = tc::named_and(kIdStore, kEpiThreads, w))) break;
             tc::tc_fence_after();
             uint8_t* xs = sm + K::OFF_X + s * K::X_BYTES;

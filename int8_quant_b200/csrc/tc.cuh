@@ -65,13 +65,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Wait for phase `parity` to complete; false if it did not within `limit` cycles.
+// Wait for phase `parity` to complete; false if it did not within `limit` cycles.  The
+// clock (and, below, the abort flag) is read once per 64 polls and not before the first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > limit) return false;
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 63) == 0 && clock64() - t0 > limit) return false;
     }
-    return true;
 }
 
 // About two seconds at the B200 boost clock: far longer than any legitimate wait here.
@@ -82,8 +84,11 @@ constexpr long long kWaitLimit = 4000000000LL;
 // status word (if any).
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               int* status, int timeout_code) {
+    if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 63) != 0) continue;
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitLimit) {
             *abort_flag = 1;
@@ -91,7 +96,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
             return false;
         }
     }
-    return true;
 }
 
 // ---------------------------------------------------------------- proxies and TMA
