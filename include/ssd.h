@@ -199,6 +199,19 @@ ssd_status ssd_calibrate_i8(const ssd_shape* shape, int prefix, const uint16_t* 
  * clears it. */
 ssd_status ssd_workspace_status(void* workspace, cudaStream_t stream);
 
+/* Self-test of the device-side bounded wait (the mechanism behind SSD_ERR_TIMEOUT):
+ * launches, on `stream`, one CTA of two warps that wait on mbarriers nothing ever
+ * completes.  Warp 0 gives up after `limit_cycles` SM clock cycles (0 < limit_cycles
+ * <= about 4e9, i.e. two seconds), raises the CTA's abort flag and records
+ * SSD_ERR_TIMEOUT in *status; warp 1, whose own limit is the kernels' full one,
+ * must leave as soon as it sees the flag.  status: device int, cleared first, then
+ * written by the kernel.  cycles: device array of 2 unsigned 64-bit counts, the
+ * cycles each warp spent waiting.  Asynchronous: returns SSD_OK once launched,
+ * SSD_ERR_INVALID_ARG for a null pointer or a limit out of range, SSD_ERR_CUDA if the
+ * launch failed.  Neither warp faults, traps or waits past its limit. */
+ssd_status ssd_selftest_bounded_wait(long long limit_cycles, int* status, unsigned long long* cycles,
+                                     cudaStream_t stream);
+
 /* Per-kernel timing (instrumentation, off by default).  While enabled, each kernel
  * the entry points enqueue is bracketed by two CUDA events on the caller's stream.
  * ssd_profile_read synchronises the recorded events and reports, for up to

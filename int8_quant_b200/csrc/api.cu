@@ -79,6 +79,8 @@ int scan_heads_per_cta(const Dims& d) {
     return best;
 }
 
+}  // namespace
+
 // The CUDA error behind this thread's last SSD_ERR_CUDA (cudaSuccess if none).
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
@@ -87,6 +89,8 @@ ssd_status from_cuda(cudaError_t e) {
     g_last_cuda_error = e;
     return SSD_ERR_CUDA;
 }
+
+namespace {
 
 #define SSD_TRY(expr)                                  \
     do {                                               \

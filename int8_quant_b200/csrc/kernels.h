@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/ssd.h"
 #include "common.cuh"
 
 namespace ssd {
@@ -109,6 +110,8 @@ cudaError_t launch_chunk_state_tc(const Dims& d, bool i8, const uint16_t* x, con
 
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
+// SSD_OK for cudaSuccess; otherwise SSD_ERR_CUDA, remembering `e` for ssd_last_cuda_error.
+ssd_status from_cuda(cudaError_t e);
 
 // Calibration helpers.
 cudaError_t launch_amax_bc(const Dims& d, const uint16_t* B, const uint16_t* C, float* amax_B,

@@ -79,18 +79,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
 // About two seconds at the B200 boost clock: far longer than any legitimate wait here.
 constexpr long long kWaitLimit = 4000000000LL;
 
-// Bounded wait of a warp-specialised kernel: gives up at once when another role has
-// raised the CTA's abort flag; on expiry raises it and records `timeout_code` in the
-// status word (if any).
+// Bounded wait of a warp-specialised kernel: gives up soon after another role has
+// raised the CTA's abort flag; on expiry (after `limit` cycles) raises it and records
+// `timeout_code` in the status word (if any).
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                              int* status, int timeout_code) {
+                                              int* status, int timeout_code, long long limit = kWaitLimit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((n & 63) != 0) continue;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimit) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             if (status) atomicExch(status, timeout_code);
             return false;

@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
 EXPORTS = ("ssd_status_string", "ssd_last_cuda_error", "ssd_workspace_bytes", "ssd_quantize_inputs", "ssd_scan_fwd_bf16",
            "ssd_scan_fwd_i8", "ssd_scan_fwd_i8_debug", "ssd_calibrate_workspace_bytes",
            "ssd_calibrate_i8", "ssd_workspace_status", "ssd_profile_enable", "ssd_profile_read",
-           "ssd_profile_reset", "ssd_scan_fwd_bf16_static")
+           "ssd_profile_reset", "ssd_scan_fwd_bf16_static", "ssd_selftest_bounded_wait")
 
 # Size of the library's fixed device scratch used by ssd_scan_fwd_bf16_static.
 STATIC_SCRATCH_BYTES = 32 << 20
@@ -92,6 +92,8 @@ def _lib():
         lib.ssd_calibrate_i8.argtypes = [sp, I, P, P, P, P, P, P, P, P, P, P, S, P]
         lib.ssd_workspace_status.restype = I
         lib.ssd_workspace_status.argtypes = [P, P]
+        lib.ssd_selftest_bounded_wait.restype = I
+        lib.ssd_selftest_bounded_wait.argtypes = [ctypes.c_longlong, P, P, P]
         lib.ssd_profile_enable.restype = I
         lib.ssd_profile_enable.argtypes = [I]
         lib.ssd_profile_reset.restype = I
@@ -189,6 +191,12 @@ def ssd_calibrate_i8(shape, prefix, x, dt, A, B, C, s_B, s_C, s_x, s_s, workspac
 
 def ssd_workspace_status(workspace, stream=None) -> int:
     return int(_lib().ssd_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def ssd_selftest_bounded_wait(limit_cycles: int, status, cycles, stream=None) -> None:
+    """status: int32 CUDA tensor of 1 element; cycles: int64 CUDA tensor of 2 elements."""
+    _check("ssd_selftest_bounded_wait", _lib().ssd_selftest_bounded_wait(
+        int(limit_cycles), _ptr(status), _ptr(cycles), _stream(stream)))
 
 
 def ssd_profile_enable(enable: bool) -> None:

@@ -99,3 +99,13 @@ def test_null_shape_is_rejected():
     assert lib.ssd_workspace_bytes(None, 0) == 0
     f = _fake()
     assert lib.ssd_scan_fwd_bf16(None, f, f, f, f, f, f, f, f, f, 1 << 20, None) == 1
+
+
+def test_bounded_wait_selftest_validates_before_any_launch():
+    lib = iq.library()
+    f = _fake()
+    assert lib.ssd_selftest_bounded_wait(0, f, f, None) == 1            # limit out of range
+    assert lib.ssd_selftest_bounded_wait(-5, f, f, None) == 1
+    assert lib.ssd_selftest_bounded_wait(1 << 40, f, f, None) == 1      # beyond the kernels' own limit
+    assert lib.ssd_selftest_bounded_wait(1000, None, f, None) == 1      # null status
+    assert lib.ssd_selftest_bounded_wait(1000, f, None, None) == 1      # null cycles
