@@ -87,10 +87,10 @@ def measured_peaks():
 NCU_TRAFFIC = {
     # batch-2 capture scaled x4 to the batch-8 launch (traffic grows with the batch);
     # see profiles/chunk_scan_tc_mamba2-2.7b-b2.md
-    ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.526592e6 + 128.723200e6),
-                                            "src_sha1": "b837bf44032720a502f416f234d9dcca352800c3"},
-    ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (270.617856e6 + 132.557056e6),
-                                            "src_sha1": "b837bf44032720a502f416f234d9dcca352800c3"},
+    ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.510976e6 + 131.441664e6),
+                                            "src_sha1": "d4289772c1f95756fab8af3deacde1b311a52d75"},
+    ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (270.597632e6 + 133.411328e6),
+                                            "src_sha1": "d4289772c1f95756fab8af3deacde1b311a52d75"},
 }
 
 
