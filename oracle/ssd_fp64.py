@@ -7,13 +7,16 @@ D [H]; head h reads group g(h) = h // (H/G) (SSDi8 notes, "background": B and C
 are stored along G and broadcast to the heads).  All arithmetic is float64.
 
 Functions and what pins them (tests/test_oracle_fp64.py):
-* ssd_sequential — the recurrence itself.  Pinned by the brute force, the
-  closed forms at L=1 and A=0, dt=0, and the hand-derived golden fixture.
-* ssd_quadratic  — y = (L∘CBᵀ)(dt⊙x) + Dx with every segment sum formed afresh.
-  Pinned against the sequential form and the golden fixture.
+* ssd_sequential — the recurrence itself, from a given initial state (zero by
+  default).  Pinned by the brute force, the closed forms at L=1 and A=0, dt=0,
+  and the hand-derived golden fixture.
+* ssd_quadratic  — y = (L∘CBᵀ)(dt⊙x) + Dx with every segment sum formed afresh,
+  plus the decayed initial state.  Pinned against the sequential form and the
+  golden fixture.
 * ssd_chunked    — ChunkCumsum, ChunkState (eq. 4 after the reconstruction),
-  StatePassing (eq. 6 read as H_{c+1} = d_c·H_c + S_c), ChunkBMM, ChunkScan1/2.
-  Pinned by chunk-size invariance against the sequential form.
+  StatePassing (eq. 6 read as H_{c+1} = d_c·H_c + S_c, H_0 the initial state),
+  ChunkBMM, ChunkScan1/2.  Pinned by chunk-size invariance against the
+  sequential form and by splitting a sequence at a chunk boundary.
 * calibrate      — static symmetric scales over a prefix.  Pinned by invariants
   (amax maps to 127, zero tensors give scale 1).
 """
@@ -55,12 +58,14 @@ def ssd_sequential(x, dt, A, B, C, D, state0=None):
     return y, h
 
 
-def ssd_quadratic(x, dt, A, B, C, D):
+def ssd_quadratic(x, dt, A, B, C, D, state0=None):
     """Brute-force "attention form" for small inputs.
 
-    y[t] = Σ_{s≤t} (C_t·B_s)·exp(Σ_{k=s+1..t} dt_k·A)·dt_s·x_s + D·x_t,
-    final = Σ_s exp(Σ_{k=s+1..L-1} dt_k·A)·dt_s·x_s ⊗ B_s.
-    Every segment sum is accumulated from scratch (no cumulative-sum differences).
+    y[t] = Σ_{s≤t} (C_t·B_s)·exp(Σ_{k=s+1..t} dt_k·A)·dt_s·x_s + D·x_t
+           + exp(Σ_{k=0..t} dt_k·A)·h0·C_t,
+    final = Σ_s exp(Σ_{k=s+1..L-1} dt_k·A)·dt_s·x_s ⊗ B_s + exp(Σ_{k=0..L-1} dt_k·A)·h0,
+    h0 the initial state (zero by default).  Every segment sum is accumulated from
+    scratch (no cumulative-sum differences).
     """
     x = np.asarray(x, np.float64)
     dt = np.asarray(dt, np.float64)
@@ -72,6 +77,7 @@ def ssd_quadratic(x, dt, A, B, C, D):
     N = Bh.shape[-1]
     y = np.empty((Bt, L, H, P))
     final = np.zeros((Bt, H, P, N))
+    h0 = None if state0 is None else np.asarray(state0, np.float64)
     for b in range(Bt):
         for h in range(H):
             a = dt[b, :, h] * A[h]
@@ -88,17 +94,28 @@ def ssd_quadratic(x, dt, A, B, C, D):
             y[b, :, h, :] = (Lmat * CB) @ u + D[h] * x[b, :, h, :]
             w = Lmat[L - 1, :] if L else np.zeros(0)       # decay from s to the end
             final[b, h] = (w[:, None] * u).T @ Bh[b, :, h, :]
+            if h0 is not None:
+                for t in range(L):
+                    acc = 0.0
+                    for k in range(t + 1):
+                        acc += a[k]
+                    y[b, t, h, :] += np.exp(acc) * (h0[b, h] @ Ch[b, t, h, :])
+                acc = 0.0
+                for k in range(L):
+                    acc += a[k]
+                final[b, h] += np.exp(acc) * h0[b, h]
     return y, final
 
 
-def ssd_chunked(x, dt, A, B, C, D, chunk: int, return_parts: bool = False, states_only: bool = False):
+def ssd_chunked(x, dt, A, B, C, D, chunk: int, return_parts: bool = False, states_only: bool = False,
+                state0=None):
     """The five SSD sub-modules in fp64, chunk length Q = `chunk`.
 
     A final partial chunk is padded with tokens of dt = 0 and x = B = C = 0,
     which leave the state and the cumulative sums unchanged.
       ChunkCumsum : Acs[j] = Σ_{i≤j} dt_i·A          (inclusive, per chunk)
       ChunkState  : S_c = Σ_j (dt_j·exp(Acs_{Q-1}-Acs_j)·x_j) ⊗ B_j   (eq. 4 with X_scaled)
-      StatePassing: H_0 = 0, H_{c+1} = exp(Acs_{Q-1})·H_c + S_c        (eq. 6)
+      StatePassing: H_0 = state0 (or 0), H_{c+1} = exp(Acs_{Q-1})·H_c + S_c   (eq. 6)
       ChunkBMM    : CB[j,i] = C_j·B_i
       ChunkScan2  : y_d[j] = Σ_{i≤j} CB[j,i]·exp(Acs_j-Acs_i)·dt_i·x_i
       ChunkScan1  : y_o[j] = exp(Acs_j)·H_c·C_j
@@ -136,6 +153,8 @@ def ssd_chunked(x, dt, A, B, C, D, chunk: int, return_parts: bool = False, state
     # StatePassing
     d = np.exp(last[:, :, 0, :])                                       # [Bt,nc,H]
     Hs = np.zeros((Bt, nc + 1, H, P, N))
+    if state0 is not None:
+        Hs[:, 0] = np.asarray(state0, np.float64)
     for c in range(nc):
         Hs[:, c + 1] = d[:, c, :, None, None] * Hs[:, c] + S[:, c]
     if states_only:

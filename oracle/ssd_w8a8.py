@@ -32,8 +32,13 @@ Readings of points the notes leave open (each also stated in the design notes):
 Parity: every integer (Bq, Cq, Xq, the INT32 accumulators, S8, H8, dq) and the
 float32 Acs are reproducible bit for bit.  Pinned by the exact-representable
 case (A = 0, dyadic inputs: the pipeline must equal the fp64 definition
-exactly), the integer-range and saturation tests, the A = 0 prefix-sum form of
-the recursion, and exp_f32's error bound against fp64 exp.  The rounding modes
+exactly, from the zero state and from a given INT8 state), the integer-range
+and saturation tests, the A = 0 prefix-sum form of the recursion, splitting a
+sequence at a chunk boundary (the second half started from the first half's
+INT8 state reproduces every integer of the whole), and exp_f32's error bound
+against fp64 exp.  `decode_step_i8` (one token on the INT8 state) is pinned
+against a one-token scan of `ssd_w8a8` (bit for bit) and, token by token on the
+exact-representable case, against the fp64 recurrence.  The rounding modes
 (half-even for rint, half-up for the shift) are this library's specification:
 parity unpinned by the notes, which do not state them.
 """
@@ -120,15 +125,18 @@ def _imatmul(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return r
 
 
-def state_passing_i8(S8: np.ndarray, dq: np.ndarray, k: int = 7) -> np.ndarray:
+def state_passing_i8(S8: np.ndarray, dq: np.ndarray, k: int = 7, init8=None) -> np.ndarray:
     """StatePassing on INT8 states (eq. 6 with S = 2^k), sequential over chunks.
 
-    S8 int8 [Bt,nc,H,P,N]; dq int [Bt,H,nc] (decay codes rint(d·2^k)).
-    H_0 = 0;  H_{c+1} = clamp(S8_c + ((dq_c·H_c + 2^(k-1)) >> k), ±127), int32 arithmetic.
+    S8 int8 [Bt,nc,H,P,N]; dq int [Bt,H,nc] (decay codes rint(d·2^k)); init8 int8
+    [Bt,H,P,N] or None (zero).
+    H_0 = init8;  H_{c+1} = clamp(S8_c + ((dq_c·H_c + 2^(k-1)) >> k), ±127), int32 arithmetic.
     Returns int8 [Bt,nc+1,H,P,N]; entry c is the state entering chunk c, entry nc the final one.
     """
     Bt, nc, H, P, N = S8.shape
     out = np.zeros((Bt, nc + 1, H, P, N), dtype=np.int8)
+    if init8 is not None:
+        out[:, 0] = np.asarray(init8, np.int8)
     half = np.int32(1 << (k - 1))
     dq = np.asarray(dq, np.int32)
     for c in range(nc):
@@ -137,8 +145,9 @@ def state_passing_i8(S8: np.ndarray, dq: np.ndarray, k: int = 7) -> np.ndarray:
     return out
 
 
-def ssd_w8a8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, chunk: int, k: int = 7) -> dict:
-    """The W8A8 SSD forward.
+def ssd_w8a8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, chunk: int, k: int = 7, init8=None) -> dict:
+    """The W8A8 SSD forward from the INT8 state init8 ([Bt,H,P,N], real value
+    init8·s_s; None is the zero state).
 
     x_vals : float32 values of the bf16 x, [Bt,L,H,P]
     dt [Bt,L,H], A [H], D [H] : float32
@@ -202,7 +211,7 @@ def ssd_w8a8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, chunk: int, k: int = 
 
     # StatePassing: fixed-point decay, multiply and shift
     dq = np.rint(exp_f32(last[..., 0]) * F32(2 ** k)).astype(np.int32)  # [Bt,H,nc]
-    H8 = state_passing_i8(S8, dq, k)                                    # [Bt,nc+1,H,P,N]
+    H8 = state_passing_i8(S8, dq, k, init8)                             # [Bt,nc+1,H,P,N]
 
     # ChunkBMM on the INT8 inputs
     CB = _imatmul(np.moveaxis(Cqp, 3, 2), np.moveaxis(Bqp, 3, 2).swapaxes(-1, -2))   # [Bt,nc,G,Q,Q]
@@ -238,3 +247,54 @@ def ssd_w8a8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, chunk: int, k: int = 
         "H8": H8[:, :nc], "CB": CB.astype(np.int32), "acc_scan1": acc_scan1.astype(np.int32),
         "lut_state": lut_state, "M": M,
     }
+
+
+def decode_step_i8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, state8, k: int = 7) -> dict:
+    """One token of the W8A8 scan on the persistent INT8 state: the chunked pipeline
+    above with a chunk of one token, so that the codes, scales and the fixed-point
+    decay are those of the scan.  With one token the chunk's cumulative sum is
+    Acs = a = dt·A, the state LUT is dt·exp(Acs - Acs) = dt (exp_f32(0) = 1), the
+    chunk decay is exp(a), CB is the single product C·B and the intra-chunk decay
+    is exp(0) = 1.
+
+    x_vals float32 values of the bf16 x [Bt,H,P]; dt [Bt,H]; A, D [H]; Bq, Cq int8
+    [Bt,G,N]; s_B, s_C [G]; s_x, s_s [H*P]; state8 int8 [Bt,H,P,N], the state before
+    the token.  Returns y float64 [Bt,H,P], state8 (after the token), and Xq, dq,
+    acc_state, S8, acc_scan1 (C·state before the token, int32 [Bt,H,P]), CB (int32 [Bt,G]).
+    """
+    x_vals = np.asarray(x_vals, F32)
+    dt = np.asarray(dt, F32)
+    A = np.asarray(A, F32)
+    D = np.asarray(D, F32)
+    Bt, H, P = x_vals.shape
+    G, N = Bq.shape[1], Bq.shape[2]
+    gh = np.arange(H) // (H // G)
+    s_B = np.asarray(s_B, F32)
+    s_C = np.asarray(s_C, F32)
+    s_x = np.asarray(s_x, F32).reshape(H, P)
+    s_s = np.asarray(s_s, F32).reshape(H, P)
+    st = np.asarray(state8, np.int8)
+
+    a = (dt * A[None, :]).astype(F32)                                   # Acs of the one-token chunk
+    lut = (dt * exp_f32((a - a).astype(F32))).astype(F32)               # LUT_state = dt·exp(0)
+    Xs = (lut[..., None] * x_vals).astype(F32)
+    Xq = quantize_sym(Xs, (F32(1.0) / s_x).astype(F32)[None])           # [Bt,H,P]
+    Bq_h = Bq[:, gh, :]                                                 # [Bt,H,N]
+    Cq_h = Cq[:, gh, :]
+    acc_state = Xq.astype(np.int64)[..., None] * Bq_h.astype(np.int64)[:, :, None, :]   # [Bt,H,P,N]
+    M = ((s_x * s_B[gh][:, None]).astype(F32) / s_s).astype(F32)
+    S8 = np.clip(np.rint(acc_state.astype(F32) * M[None, :, :, None]), -QMAX, QMAX).astype(np.int8)
+    dq = np.rint(exp_f32(a) * F32(2 ** k)).astype(np.int32)             # [Bt,H]
+    carried = (dq[:, :, None, None] * st.astype(np.int32) + np.int32(1 << (k - 1))) >> np.int32(k)
+    new8 = np.clip(S8.astype(np.int32) + carried, -QMAX, QMAX).astype(np.int8)
+
+    acc1 = np.einsum("bhpn,bhn->bhp", st.astype(np.int64), Cq_h.astype(np.int64))      # ChunkScan1
+    CB = np.einsum("bgn,bgn->bg", Cq.astype(np.int64), Bq.astype(np.int64))            # ChunkBMM
+    f64 = np.float64
+    y_o = acc1.astype(f64) * (s_C.astype(f64)[gh][:, None] * s_s.astype(f64))[None] \
+        * np.exp(a.astype(f64))[..., None]
+    y_d = CB[:, gh].astype(f64)[..., None] * (s_C.astype(f64) * s_B.astype(f64))[gh][None, :, None] \
+        * dt.astype(f64)[..., None] * x_vals.astype(f64)
+    y = y_o + y_d + D.astype(f64)[None, :, None] * x_vals.astype(f64)
+    return {"y": y, "state8": new8, "Xq": Xq, "dq": dq, "acc_state": acc_state.astype(np.int32), "S8": S8,
+            "acc_scan1": acc1.astype(np.int32), "CB": CB.astype(np.int32)}

@@ -198,3 +198,64 @@ def test_calibrate_invariants():
     np.testing.assert_allclose(amax / sc["s_x"].astype(np.float64), 127.0, rtol=1e-6)
     z = F.calibrate(0 * x, dt, A, 0 * B, 0 * C, chunk=64)
     assert np.all(z["s_B"] == 1) and np.all(z["s_x"] == 1) and np.all(z["s_s"] == 1)
+
+
+# ---------------------------------------------------------------- initial state
+def _state0(seed, Bt, H, P, N):
+    return np.random.default_rng(100 + seed).standard_normal((Bt, H, P, N))
+
+
+@pytest.mark.parametrize("L", [1, 2, 7, 64])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_initial_state_sequential_equals_bruteforce(L, seed):
+    args = _inputs(seed, 2, L, 4, 3, 5, 2)
+    h0 = _state0(seed, 2, 4, 3, 5)
+    ys, fs = F.ssd_sequential(*args, state0=h0)
+    yq, fq = F.ssd_quadratic(*args, state0=h0)
+    assert rel_l2(ys, yq) < 1e-12 and rel_l2(fs, fq) < 1e-12
+    # the initial state really enters: both forms differ from the zero-state result
+    y0, _ = F.ssd_sequential(*args)
+    assert rel_l2(ys, y0) > 1e-3
+
+
+def test_initial_state_is_linear_superposition():
+    # the recurrence is linear in the state: y(h0) = y(0) + (decayed h0)·C
+    x, dt, A, B, C, D = _inputs(3, 1, 9, 2, 3, 4, 1)
+    h0 = _state0(3, 1, 2, 3, 4)
+    y, fin = F.ssd_sequential(x, dt, A, B, C, D, state0=h0)
+    y0, fin0 = F.ssd_sequential(x, dt, A, B, C, D)
+    acs = np.cumsum(dt * A[None, None, :], axis=1)                        # Σ_{k≤t} a_k   [1,L,H]
+    Ch = C[:, :, np.arange(2) // 2]
+    extra = np.exp(acs)[..., None] * np.einsum("bhpn,blhn->blhp", h0, Ch)
+    assert rel_l2(y, y0 + extra) < 1e-12
+    assert rel_l2(fin, fin0 + np.exp(acs[:, -1])[..., None, None] * h0) < 1e-12
+
+
+@pytest.mark.parametrize("Q", [16, 64])
+def test_initial_state_chunked_equals_sequential(Q):
+    args = _inputs(4, 2, 150, 4, 3, 5, 2)
+    h0 = _state0(4, 2, 4, 3, 5)
+    ys, fs = F.ssd_sequential(*args, state0=h0)
+    yc, fc = F.ssd_chunked(*args, chunk=Q, state0=h0)
+    assert rel_l2(yc, ys) < 1e-12 and rel_l2(fc, fs) < 1e-12
+
+
+def test_split_at_a_chunk_boundary_equals_the_whole():
+    x, dt, A, B, C, D = _inputs(8, 2, 192, 4, 3, 5, 2)
+    y, fin = F.ssd_chunked(x, dt, A, B, C, D, chunk=64)
+    y1, f1 = F.ssd_chunked(x[:, :128], dt[:, :128], A, B[:, :128], C[:, :128], D, chunk=64)
+    y2, f2 = F.ssd_chunked(x[:, 128:], dt[:, 128:], A, B[:, 128:], C[:, 128:], D, chunk=64, state0=f1)
+    assert rel_l2(np.concatenate([y1, y2], axis=1), y) < 1e-12
+    assert rel_l2(f2, fin) < 1e-12
+
+
+def test_A_zero_with_initial_state_closed_form():
+    x, dt, A, B, C, D = _inputs(9, 2, 40, 4, 3, 5, 2)
+    A0 = np.zeros_like(A)
+    h0 = _state0(9, 2, 4, 3, 5)
+    y, fin = F.ssd_sequential(x, dt, A0, B, C, D, state0=h0)
+    g = np.arange(4) // 2
+    inject = (dt[..., None] * x)[..., None] * B[:, :, g][:, :, :, None, :]
+    h = h0[:, None] + np.cumsum(inject, axis=1)                           # h_t = h0 + Σ_{s≤t} dt x Bᵀ
+    ey = np.einsum("blhpn,blhn->blhp", h, C[:, :, g]) + D[None, None, :, None] * x
+    assert rel_l2(y, ey) < 1e-12 and rel_l2(fin, h[:, -1]) < 1e-12

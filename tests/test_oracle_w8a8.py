@@ -188,3 +188,81 @@ def test_w8a8_output_within_tolerance_of_fp64(name):
                    w.chunk)
     ys, _ = F.ssd_sequential(x, d["dt"], d["A"], Bv, Cv, d["D"])
     assert rel_l2(r["y"], ys) <= 5e-2
+
+
+# ---------------------------------------------------------------- initial state and decode step
+def _calibrated(w, prefix=64):
+    d = make_inputs(w)
+    x, Bv, Cv = as_float(d["x"]).astype(F32), as_float(d["B"]).astype(F32), as_float(d["C"]).astype(F32)
+    sc = F.calibrate(x, d["dt"], d["A"], Bv, Cv, w.chunk, prefix=prefix)
+    Bq, Cq = W.quantize_inputs(Bv, Cv, sc["s_B"], sc["s_C"])
+    return d, x, Bq, Cq, sc
+
+
+def test_w8a8_split_at_a_chunk_boundary_is_bit_exact():
+    w = Workload("t", 2, 320, 4, 8, 16, 2, 64, seed=11, head_scale=True, outliers=True)
+    d, x, Bq, Cq, sc = _calibrated(w)
+    args = (d["A"], d["D"], sc["s_B"], sc["s_C"], sc["s_x"], sc["s_s"], 64)
+    whole = W.ssd_w8a8(x, d["dt"], Bq=Bq, Cq=Cq, **dict(zip(("A", "D", "s_B", "s_C", "s_x", "s_s", "chunk"), args)))
+    cut = 192
+    kw = dict(zip(("A", "D", "s_B", "s_C", "s_x", "s_s", "chunk"), args))
+    r1 = W.ssd_w8a8(x[:, :cut], d["dt"][:, :cut], Bq=Bq[:, :cut], Cq=Cq[:, :cut], **kw)
+    r2 = W.ssd_w8a8(x[:, cut:], d["dt"][:, cut:], Bq=Bq[:, cut:], Cq=Cq[:, cut:], init8=r1["final8"], **kw)
+    assert (r1["final8"] != 0).any(), "the carried state must be non-trivial"
+    np.testing.assert_array_equal(np.concatenate([r1["H8"], r2["H8"]], axis=1), whole["H8"])
+    np.testing.assert_array_equal(np.concatenate([r1["S8"], r2["S8"]], axis=1), whole["S8"])
+    np.testing.assert_array_equal(np.concatenate([r1["acc_scan1"], r2["acc_scan1"]], axis=1), whole["acc_scan1"])
+    np.testing.assert_array_equal(r2["final8"], whole["final8"])
+    np.testing.assert_array_equal(np.concatenate([r1["y"], r2["y"]], axis=1), whole["y"])
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_w8a8_with_initial_state_equals_fp64_exactly_when_representable(seed):
+    x, dt, A, Bv, Cv, D, s_B, s_C, s_x, s_s, Q = _exact_case(seed)
+    Bq, Cq = W.quantize_inputs(Bv, Cv, s_B, s_C)
+    Bt, L, H, P = x.shape
+    init8 = np.random.default_rng(50 + seed).integers(-20, 21, (Bt, H, P, Bv.shape[-1])).astype(np.int8)
+    r = W.ssd_w8a8(x, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, Q, init8=init8)
+    assert np.abs(r["final8"]).max() < 127, "case must not saturate"
+    h0 = init8.astype(np.float64) * s_s.reshape(H, P)[None, :, :, None].astype(np.float64)
+    ys, fs = F.ssd_sequential(x, dt, A, Bv, Cv, D, state0=h0)
+    np.testing.assert_allclose(r["y"], ys, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["final"], fs, rtol=0, atol=1e-12)
+
+
+def test_decode_step_equals_a_one_token_scan():
+    w = Workload("t", 2, 257, 4, 8, 16, 2, 64, seed=12, head_scale=True, outliers=True)
+    d, x, Bq, Cq, sc = _calibrated(w)
+    kw = dict(A=d["A"], D=d["D"], s_B=sc["s_B"], s_C=sc["s_C"], s_x=sc["s_x"], s_s=sc["s_s"])
+    r0 = W.ssd_w8a8(x[:, :256], d["dt"][:, :256], Bq=Bq[:, :256], Cq=Cq[:, :256], chunk=64, **kw)
+    t = 256
+    step = W.decode_step_i8(x[:, t], d["dt"][:, t], Bq=Bq[:, t], Cq=Cq[:, t], state8=r0["final8"], **kw)
+    one = W.ssd_w8a8(x[:, t:t + 1], d["dt"][:, t:t + 1], Bq=Bq[:, t:t + 1], Cq=Cq[:, t:t + 1], chunk=32,
+                     init8=r0["final8"], **kw)
+    np.testing.assert_array_equal(step["state8"], one["final8"])
+    np.testing.assert_array_equal(step["Xq"], one["Xq"][:, 0])
+    np.testing.assert_array_equal(step["S8"], one["S8"][:, 0])
+    np.testing.assert_array_equal(step["acc_state"], one["acc_state"][:, 0])
+    np.testing.assert_array_equal(step["dq"], one["dq"][:, :, 0])
+    np.testing.assert_array_equal(step["acc_scan1"], one["acc_scan1"][:, 0])
+    np.testing.assert_array_equal(step["CB"], one["CB"][:, 0, :, 0, 0])
+    np.testing.assert_allclose(step["y"], one["y"][:, 0], rtol=1e-13, atol=1e-12)
+    # the scan over all 257 tokens (the last one alone in a padded chunk) ends in the same state
+    full = W.ssd_w8a8(x, d["dt"], Bq=Bq, Cq=Cq, chunk=64, **kw)
+    np.testing.assert_array_equal(full["final8"], step["state8"])
+    assert not np.array_equal(step["state8"], r0["final8"])
+
+
+def test_decode_steps_equal_fp64_exactly_when_representable():
+    x, dt, A, Bv, Cv, D, s_B, s_C, s_x, s_s, Q = _exact_case(3, L=24)
+    Bq, Cq = W.quantize_inputs(Bv, Cv, s_B, s_C)
+    Bt, L, H, P = x.shape
+    N = Bv.shape[-1]
+    st = np.zeros((Bt, H, P, N), np.int8)
+    ys, fs = F.ssd_sequential(x, dt, A, Bv, Cv, D)
+    for t in range(L):
+        r = W.decode_step_i8(x[:, t], dt[:, t], A, Bq[:, t], Cq[:, t], D, s_B, s_C, s_x, s_s, st)
+        np.testing.assert_allclose(r["y"], ys[:, t], rtol=0, atol=1e-12)
+        st = r["state8"]
+    assert np.abs(st).max() < 127
+    np.testing.assert_allclose(st.astype(np.float64) * s_s.reshape(H, P)[None, :, :, None], fs, rtol=0, atol=1e-12)
