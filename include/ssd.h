@@ -140,6 +140,18 @@ ssd_status ssd_scan_fwd_bf16_static(const ssd_shape* shape, const uint16_t* x, c
                                     const float* D, uint16_t* y, float* final_state,
                                     cudaStream_t stream);
 
+/* ssd_scan_fwd_bf16 continuing from a given state: h_{-1} = initial_state (device fp32
+ * [B, H, P, N], 16-byte aligned; null means zero, as in ssd_scan_fwd_bf16).  Feeding
+ * a call's final_state to the next call over the following tokens reproduces one
+ * call over both (bit for bit when the split falls on a chunk boundary).  With
+ * seqlen 0, final_state receives a copy of initial_state.  The initial state enters
+ * StatePassing as H_0 ("SSDi8" notes, eq. 6); everything else is unchanged. */
+ssd_status ssd_scan_fwd_bf16_from_state(const ssd_shape* shape, const uint16_t* x, const float* dt,
+                                        const float* A, const uint16_t* B, const uint16_t* C,
+                                        const float* D, const float* initial_state, uint16_t* y,
+                                        float* final_state, void* workspace, size_t workspace_bytes,
+                                        cudaStream_t stream);
+
 /* W8A8 SSD forward on the INT8 inputs of ssd_quantize_inputs.
  * x, dt, A, D, y : as in ssd_scan_fwd_bf16.   Bq, Cq : device int8 [B, L, G, N].
  * params : host pointer to the scales (device arrays) and the decay shift k.
@@ -172,6 +184,17 @@ typedef struct {
     int32_t* cb;
     int32_t* acc_scan1;
 } ssd_i8_debug;
+
+/* ssd_scan_fwd_i8 continuing from a given INT8 state: initial_state is device int8
+ * [B, H, P, N] in the same codes as final_state (real value = code * s_s[h*P+p]),
+ * 16-byte aligned; null means zero.  It is H_0 of the integer StatePassing (eq. 6),
+ * so a call's final_state fed to the call over the following tokens reproduces
+ * every integer of one call over both when the split falls on a chunk boundary. */
+ssd_status ssd_scan_fwd_i8_from_state(const ssd_shape* shape, const uint16_t* x, const float* dt,
+                                      const float* A, const int8_t* Bq, const int8_t* Cq, const float* D,
+                                      const ssd_i8_params* params, const int8_t* initial_state, uint16_t* y,
+                                      int8_t* final_state, void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream);
 
 /* ssd_scan_fwd_i8 that also writes the intermediates named in `dbg` (host pointer). */
 ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, const float* dt,

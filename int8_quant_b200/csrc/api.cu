@@ -234,20 +234,23 @@ static ssd_status check_common(const Dims& d, const void* x, const float* dt, co
     return SSD_OK;
 }
 
-ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const float* dt,
-                             const float* A, const uint16_t* B, const uint16_t* C,
-                             const float* D, uint16_t* y, float* final_state, void* workspace,
-                             size_t workspace_bytes, cudaStream_t stream) {
+static ssd_status scan_bf16(const ssd_shape* shape, const uint16_t* x, const float* dt, const float* A,
+                            const uint16_t* B, const uint16_t* C, const float* D, const float* initial_state,
+                            uint16_t* y, float* final_state, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
     Dims d;
     ssd_status st = make_dims(shape, &d);
     if (st != SSD_OK) return st;
     if (d.B == 0) return SSD_OK;
     st = check_common(d, x, dt, A, B, C, D, y, final_state, workspace, workspace_bytes, false);
     if (st != SSD_OK) return st;
+    if (initial_state && !aligned16(initial_state)) return SSD_ERR_INVALID_ARG;
     const size_t fs_bytes = (size_t)d.B * d.H * d.P * d.N * sizeof(float);
     const WsLayout w = ws_layout(d, false);
     if (d.L == 0) {
         SSD_TRY(cudaMemsetAsync(at<int>(workspace, w.status), 0, sizeof(int), stream));
+        if (initial_state)
+            return from_cuda(cudaMemcpyAsync(final_state, initial_state, fs_bytes, cudaMemcpyDeviceToDevice, stream));
         return from_cuda(cudaMemsetAsync(final_state, 0, fs_bytes, stream));
     }
     float* Acs = at<float>(workspace, w.acs);
@@ -266,7 +269,8 @@ ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const fl
     else
         SSD_STAGE("chunk_state", launch_chunk_state_bf16(d, x, dt, Acs, B, static_cast<float*>(S), nullptr, nullptr,
                                                          stream));
-    SSD_STAGE("state_passing", launch_state_passing_bf16(d, S, !tcs, decay, Hc, final_state, nullptr, stream));
+    SSD_STAGE("state_passing",
+              launch_state_passing_bf16(d, S, !tcs, decay, initial_state, Hc, final_state, nullptr, stream));
     if (tensor_core_shape(d))
         SSD_STAGE("chunk_scan", launch_chunk_scan_tc(d, false, x, B, C, Acs, dtc, D, I8Scales{}, Hc, y, nullptr,
                                                      scan_heads_per_cta(d), status, stream));
@@ -275,11 +279,25 @@ ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const fl
     return SSD_OK;
 }
 
-ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, const float* dt,
-                                 const float* A, const int8_t* Bq, const int8_t* Cq,
-                                 const float* D, const ssd_i8_params* params, uint16_t* y,
-                                 int8_t* final_state, void* workspace, size_t workspace_bytes,
-                                 const ssd_i8_debug* dbg, cudaStream_t stream) {
+ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const float* dt,
+                             const float* A, const uint16_t* B, const uint16_t* C,
+                             const float* D, uint16_t* y, float* final_state, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
+    return scan_bf16(shape, x, dt, A, B, C, D, nullptr, y, final_state, workspace, workspace_bytes, stream);
+}
+
+ssd_status ssd_scan_fwd_bf16_from_state(const ssd_shape* shape, const uint16_t* x, const float* dt,
+                                        const float* A, const uint16_t* B, const uint16_t* C,
+                                        const float* D, const float* initial_state, uint16_t* y,
+                                        float* final_state, void* workspace, size_t workspace_bytes,
+                                        cudaStream_t stream) {
+    return scan_bf16(shape, x, dt, A, B, C, D, initial_state, y, final_state, workspace, workspace_bytes, stream);
+}
+
+static ssd_status scan_i8(const ssd_shape* shape, const uint16_t* x, const float* dt, const float* A,
+                          const int8_t* Bq, const int8_t* Cq, const float* D, const ssd_i8_params* params,
+                          const int8_t* initial_state, uint16_t* y, int8_t* final_state, void* workspace,
+                          size_t workspace_bytes, const ssd_i8_debug* dbg, cudaStream_t stream) {
     Dims d;
     ssd_status st = make_dims(shape, &d);
     if (st != SSD_OK) return st;
@@ -288,10 +306,13 @@ ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, cons
     if (d.B == 0) return SSD_OK;
     st = check_common(d, x, dt, A, Bq, Cq, D, y, final_state, workspace, workspace_bytes, true);
     if (st != SSD_OK) return st;
+    if (initial_state && !aligned16(initial_state)) return SSD_ERR_INVALID_ARG;
     const size_t fs_bytes = (size_t)d.B * d.H * d.P * d.N;
     const WsLayout w = ws_layout(d, true);
     if (d.L == 0) {
         SSD_TRY(cudaMemsetAsync(at<int>(workspace, w.status), 0, sizeof(int), stream));
+        if (initial_state)
+            return from_cuda(cudaMemcpyAsync(final_state, initial_state, fs_bytes, cudaMemcpyDeviceToDevice, stream));
         return from_cuda(cudaMemsetAsync(final_state, 0, fs_bytes, stream));
     }
     float* Acs = at<float>(workspace, w.acs);
@@ -312,7 +333,7 @@ ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, cons
                                                        status, stream));
     else
         SSD_STAGE("chunk_state", launch_chunk_state_i8(d, x, dt, Acs, Bq, sc, S8, dbg ? &dd : nullptr, stream));
-    SSD_STAGE("state_passing", launch_state_passing_i8(d, S8, dq, sc.shift, H8, final_state, stream));
+    SSD_STAGE("state_passing", launch_state_passing_i8(d, S8, dq, sc.shift, initial_state, H8, final_state, stream));
     if (tensor_core_shape(d))
         SSD_STAGE("chunk_scan", launch_chunk_scan_tc(d, true, x, Bq, Cq, Acs, dtc, D, sc, H8, y, dbg ? &dd : nullptr,
                                                      scan_heads_per_cta(d), status, stream));
@@ -328,12 +349,30 @@ ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, cons
     return SSD_OK;
 }
 
+ssd_status ssd_scan_fwd_i8_debug(const ssd_shape* shape, const uint16_t* x, const float* dt,
+                                 const float* A, const int8_t* Bq, const int8_t* Cq,
+                                 const float* D, const ssd_i8_params* params, uint16_t* y,
+                                 int8_t* final_state, void* workspace, size_t workspace_bytes,
+                                 const ssd_i8_debug* dbg, cudaStream_t stream) {
+    return scan_i8(shape, x, dt, A, Bq, Cq, D, params, nullptr, y, final_state, workspace, workspace_bytes, dbg,
+                   stream);
+}
+
 ssd_status ssd_scan_fwd_i8(const ssd_shape* shape, const uint16_t* x, const float* dt,
                            const float* A, const int8_t* Bq, const int8_t* Cq, const float* D,
                            const ssd_i8_params* params, uint16_t* y, int8_t* final_state,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-    return ssd_scan_fwd_i8_debug(shape, x, dt, A, Bq, Cq, D, params, y, final_state, workspace,
-                                 workspace_bytes, nullptr, stream);
+    return scan_i8(shape, x, dt, A, Bq, Cq, D, params, nullptr, y, final_state, workspace, workspace_bytes, nullptr,
+                   stream);
+}
+
+ssd_status ssd_scan_fwd_i8_from_state(const ssd_shape* shape, const uint16_t* x, const float* dt,
+                                      const float* A, const int8_t* Bq, const int8_t* Cq, const float* D,
+                                      const ssd_i8_params* params, const int8_t* initial_state, uint16_t* y,
+                                      int8_t* final_state, void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream) {
+    return scan_i8(shape, x, dt, A, Bq, Cq, D, params, initial_state, y, final_state, workspace, workspace_bytes,
+                   nullptr, stream);
 }
 
 static WsLayout calib_layout(const Dims& p, size_t* fin_off, size_t* amax_off) {
@@ -390,7 +429,7 @@ ssd_status ssd_calibrate_i8(const ssd_shape* shape, int prefix, const uint16_t* 
         SSD_TRY(launch_amax_bc(p, B, C, aB, aC, stream));
         SSD_TRY(launch_cumsum(p, dt, A, Acs, decay, nullptr, 0, nullptr, nullptr, nullptr, stream));
         SSD_TRY(launch_chunk_state_bf16(p, x, dt, Acs, B, S, ax, as, stream));
-        SSD_TRY(launch_state_passing_bf16(p, S, true, decay, nullptr, fin, ah, stream));
+        SSD_TRY(launch_state_passing_bf16(p, S, true, decay, nullptr, nullptr, fin, ah, stream));
     }
     SSD_TRY(launch_amax_to_scale(aB, 2 * d.G + d.H * d.P, stream));       // s_B, s_C, s_x
     SSD_TRY(launch_amax_pair_to_scale(as, ah, s_s, d.H * d.P, stream));    // s_s over S and H

@@ -65,11 +65,12 @@ cudaError_t launch_chunk_state_i8(const Dims& d, const uint16_t* x, const float*
 //   bf16: H_{c+1} = decay_c * H_c + S_c in fp32; writes the state entering each
 //         chunk as bf16 (Hc) and/or fp32 (Hc32), the final state as fp32.
 //   W8A8: H_{c+1} = sat127(S8_c + ((dq_c * H_c + 2^(k-1)) >> k)).
+// init (fp32 [B,H,P,N]) / init8 (INT8 codes [B,H,P,N]): the state before the first chunk, or null for zero.
 cudaError_t launch_state_passing_bf16(const Dims& d, const void* S, bool s_fp32, const float* decay,
-                                      uint16_t* Hc, float* final_state, float* amax_h,
+                                      const float* init, uint16_t* Hc, float* final_state, float* amax_h,
                                       cudaStream_t st);
 cudaError_t launch_state_passing_i8(const Dims& d, const int8_t* S8, const int32_t* dq, int shift,
-                                    int8_t* H8, int8_t* final_state, cudaStream_t st);
+                                    const int8_t* init8, int8_t* H8, int8_t* final_state, cudaStream_t st);
 
 // a4-a7: ChunkBMM + ChunkScan2 (diagonal) + ChunkScan1 (off-diagonal) + D skip.
 cudaError_t launch_chunk_scan_bf16(const Dims& d, const uint16_t* x, const float* dt,

@@ -1,6 +1,7 @@
 // state_passing.cu — a3, StatePassing (SSDi8 notes, eq. 6), sequential over chunks.
-//   bf16 : H_0 = 0, H_{c+1} = exp(Acs_c[Q-1]) * H_c + S_c  (fp32; S_c stored as bf16)
+//   bf16 : H_{c+1} = exp(Acs_c[Q-1]) * H_c + S_c  (fp32; S_c stored as bf16)
 //   W8A8 : H_{c+1} = sat127(S8_c + ((dq_c * H_c + 2^(k-1)) >> k))       (int32, then INT8)
+// H_0 is the caller's initial state (fp32, or INT8 codes in the s_s scales), or zero.
 // Every (p,n) element of a (b,h) state is an independent scalar recurrence, so one
 // thread owns 4 (bf16 path) or 16 (W8A8) consecutive elements and walks the chunks; consecutive threads own
 // consecutive elements (coalesced vector loads and stores).  Loads of the next
@@ -32,7 +33,8 @@ __device__ __forceinline__ F4 load4(const uint16_t* p) {
 template <typename TS>
 __global__ void __launch_bounds__(kThreads)
 state_passing_bf16_kernel(Dims d, const TS* __restrict__ S, const float* __restrict__ decay,
-                          uint16_t* __restrict__ Hc, float* __restrict__ final_state, float* amax_h) {
+                          const float* __restrict__ init, uint16_t* __restrict__ Hc, float* __restrict__ final_state,
+                          float* amax_h) {
     const int PN = d.P * d.N;
     const int e = (blockIdx.x * kThreads + threadIdx.x) * kVec;
     const int h = blockIdx.y, b = blockIdx.z;
@@ -42,6 +44,11 @@ state_passing_bf16_kernel(Dims d, const TS* __restrict__ S, const float* __restr
     uint16_t* hc = Hc ? Hc + ((long long)b * d.nc * d.H + h) * PN + e : nullptr;
     const float* dec = decay + ((long long)b * d.H + h) * d.nc;
     float hv[kVec] = {0.f, 0.f, 0.f, 0.f};
+    if (init) {
+        const F4 h0 = load4(init + ((long long)b * d.H + h) * PN + e);
+#pragma unroll
+        for (int v = 0; v < kVec; ++v) hv[v] = h0.v[v];
+    }
     float amax = 0.f;
     for (int c0 = 0; c0 < d.nc; c0 += kAhead) {
         F4 sv[kAhead];
@@ -76,7 +83,8 @@ constexpr int kVecI8 = 16;                               // INT8 elements per th
 
 __global__ void __launch_bounds__(kThreads)
 state_passing_i8_kernel(Dims d, const int8_t* __restrict__ S8, const int32_t* __restrict__ dq,
-                        int shift, int8_t* __restrict__ H8, int8_t* __restrict__ final_state) {
+                        int shift, const int8_t* __restrict__ init8, int8_t* __restrict__ H8,
+                        int8_t* __restrict__ final_state) {
     const int PN = d.P * d.N;
     const int e = (blockIdx.x * kThreads + threadIdx.x) * kVecI8;
     const int h = blockIdx.y, b = blockIdx.z;
@@ -89,6 +97,12 @@ state_passing_i8_kernel(Dims d, const int8_t* __restrict__ S8, const int32_t* __
     int hv[kVecI8];
 #pragma unroll
     for (int v = 0; v < kVecI8; ++v) hv[v] = 0;
+    if (init8) {
+        const uint4 t = __ldg(reinterpret_cast<const uint4*>(init8 + ((long long)b * d.H + h) * PN + e));
+        const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int v = 0; v < kVecI8; ++v) hv[v] = (int)(int8_t)(w[v >> 2] >> (8 * (v & 3)));
+    }
     auto pack = [&]() -> uint4 {
         uint32_t w[4];
 #pragma unroll
@@ -127,26 +141,26 @@ state_passing_i8_kernel(Dims d, const int8_t* __restrict__ S8, const int32_t* __
 }  // namespace
 
 cudaError_t launch_state_passing_bf16(const Dims& d, const void* S, bool s_fp32, const float* decay,
-                                      uint16_t* Hc, float* final_state, float* amax_h,
+                                      const float* init, uint16_t* Hc, float* final_state, float* amax_h,
                                       cudaStream_t st) {
     if (d.B == 0) return cudaSuccess;
     if ((d.P * d.N) % kVec != 0 || d.N % kVec != 0) return cudaErrorInvalidValue;
     dim3 grid((d.P * d.N / kVec + kThreads - 1) / kThreads, d.H, d.B);
     if (s_fp32)
-        state_passing_bf16_kernel<float><<<grid, kThreads, 0, st>>>(d, static_cast<const float*>(S), decay, Hc,
-                                                                     final_state, amax_h);
+        state_passing_bf16_kernel<float><<<grid, kThreads, 0, st>>>(d, static_cast<const float*>(S), decay, init,
+                                                                     Hc, final_state, amax_h);
     else
         state_passing_bf16_kernel<uint16_t><<<grid, kThreads, 0, st>>>(d, static_cast<const uint16_t*>(S), decay,
-                                                                        Hc, final_state, amax_h);
+                                                                        init, Hc, final_state, amax_h);
     return cudaGetLastError();
 }
 
 cudaError_t launch_state_passing_i8(const Dims& d, const int8_t* S8, const int32_t* dq, int shift,
-                                    int8_t* H8, int8_t* final_state, cudaStream_t st) {
+                                    const int8_t* init8, int8_t* H8, int8_t* final_state, cudaStream_t st) {
     if (d.B == 0) return cudaSuccess;
     if ((d.P * d.N) % kVecI8 != 0) return cudaErrorInvalidValue;
     dim3 grid((d.P * d.N / kVecI8 + kThreads - 1) / kThreads, d.H, d.B);
-    state_passing_i8_kernel<<<grid, kThreads, 0, st>>>(d, S8, dq, shift, H8, final_state);
+    state_passing_i8_kernel<<<grid, kThreads, 0, st>>>(d, S8, dq, shift, init8, H8, final_state);
     return cudaGetLastError();
 }
 

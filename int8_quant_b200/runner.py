@@ -52,10 +52,15 @@ class SsdProblem:
         self.params = None
 
     # -- bf16
-    def run_bf16(self, stream=None):
+    def run_bf16(self, stream=None, initial_state=None):
+        """initial_state: fp32 [B,H,P,N] device tensor to continue from (None: zero state)."""
         i = self.inp
-        ssd.ssd_scan_fwd_bf16(self.shape, i["x"], i["dt"], i["A"], i["B"], i["C"], i["D"], self.y,
-                              self.final32, self.ws_bf16, stream)
+        if initial_state is None:
+            ssd.ssd_scan_fwd_bf16(self.shape, i["x"], i["dt"], i["A"], i["B"], i["C"], i["D"], self.y,
+                                  self.final32, self.ws_bf16, stream)
+        else:
+            ssd.ssd_scan_fwd_bf16_from_state(self.shape, i["x"], i["dt"], i["A"], i["B"], i["C"], i["D"],
+                                             initial_state, self.y, self.final32, self.ws_bf16, stream)
 
     # -- W8A8
     def set_scales(self, s_B, s_C, s_x, s_s, shift: int = 7):
@@ -84,12 +89,17 @@ class SsdProblem:
         ssd.ssd_quantize_inputs(self.shape, i["B"], i["C"], self.scales["s_B"], self.scales["s_C"], self.Bq,
                                 self.Cq, stream)
 
-    def run_i8(self, stream=None, quantize=True):
+    def run_i8(self, stream=None, quantize=True, initial_state=None):
+        """initial_state: int8 [B,H,P,N] device tensor of state codes (None: zero state)."""
         if quantize:
             self.quantize(stream)
         i = self.inp
-        ssd.ssd_scan_fwd_i8(self.shape, i["x"], i["dt"], i["A"], self.Bq, self.Cq, i["D"], self.params, self.y,
-                            self.final8, self.ws_i8, stream)
+        if initial_state is None:
+            ssd.ssd_scan_fwd_i8(self.shape, i["x"], i["dt"], i["A"], self.Bq, self.Cq, i["D"], self.params, self.y,
+                                self.final8, self.ws_i8, stream)
+        else:
+            ssd.ssd_scan_fwd_i8_from_state(self.shape, i["x"], i["dt"], i["A"], self.Bq, self.Cq, i["D"],
+                                           self.params, initial_state, self.y, self.final8, self.ws_i8, stream)
 
     def run_i8_debug(self, stream=None):
         b, L, H, P, G, N, Q = self.dims
