@@ -222,6 +222,34 @@ ssd_status ssd_calibrate_i8(const ssd_shape* shape, int prefix, const uint16_t* 
  * clears it. */
 ssd_status ssd_workspace_status(void* workspace, cudaStream_t stream);
 
+/* One token on the persistent state, in place (serving: the step after a scan, whose
+ * final_state it continues; the recurrence the SSD factorises, one token at a time):
+ *   h <- exp(dt*A) * h + dt * x B^T,      y = C . h + D * x
+ * shape: batch, nheads, headdim, ngroups, dstate as in the scan; seqlen must be 1;
+ *   chunk is not used.  Supported (P, N) as in the scan.
+ * x  : device bf16 [B, H, P]          dt : device fp32 [B, H]
+ * A, D : device fp32 [H]              B, C : device bf16 [B, G, N]
+ * state : device fp32 [B, H, P, N], read and overwritten (the scan's final_state format)
+ * y  : device bf16 [B, H, P], written.
+ * All pointers 16-byte aligned.  Argument errors return before any launch. */
+ssd_status ssd_decode_step_bf16(const ssd_shape* shape, const uint16_t* x, const float* dt, const float* A,
+                                const uint16_t* B, const uint16_t* C, const float* D, float* state, uint16_t* y,
+                                cudaStream_t stream);
+
+/* W8A8 one-token step on the INT8 state of ssd_scan_fwd_i8 (codes, real value code *
+ * s_s[h*P+p]), in place: the scan's integer steps with a chunk of one token ("SSDi8"
+ * notes, key designs 1-2, eq. 6), so that the state codes equal those of
+ * ssd_scan_fwd_i8_from_state over that token:
+ *   a = dt*A;  Xq = clamp(rint(dt*x / s_x));  S8 = clamp(rint((Xq*Bq) * (s_x*s_B/s_s)))
+ *   dq = rint(exp(a) * 2^k);  H <- sat127(S8 + ((dq*H + 2^(k-1)) >> k))
+ *   y = (Cq.H_before)*s_C*s_s*exp(a) + (Cq.Bq)*s_C*s_B*dt*x + D*x     (bf16)
+ * Bq, Cq : device int8 [B, G, N] (ssd_quantize_inputs with seqlen 1).  params as in
+ * ssd_scan_fwd_i8.  state : device int8 [B, H, P, N], read and overwritten.  Other
+ * arguments as in ssd_decode_step_bf16. */
+ssd_status ssd_decode_step_i8(const ssd_shape* shape, const uint16_t* x, const float* dt, const float* A,
+                              const int8_t* Bq, const int8_t* Cq, const float* D, const ssd_i8_params* params,
+                              int8_t* state, uint16_t* y, cudaStream_t stream);
+
 /* Self-test of the device-side bounded wait (the mechanism behind SSD_ERR_TIMEOUT):
  * launches, on `stream`, one CTA of two warps that wait on mbarriers nothing ever
  * completes.  Warp 0 gives up after `limit_cycles` SM clock cycles (0 < limit_cycles

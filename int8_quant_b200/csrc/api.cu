@@ -375,6 +375,51 @@ ssd_status ssd_scan_fwd_i8_from_state(const ssd_shape* shape, const uint16_t* x,
                    nullptr, stream);
 }
 
+// Shape of a one-token step: seqlen must be 1; chunk is not used.
+static ssd_status decode_dims(const ssd_shape* s, Dims* d) {
+    if (!s) return SSD_ERR_INVALID_ARG;
+    if (s->batch < 0 || s->seqlen != 1 || s->nheads < 1 || s->ngroups < 1 || s->headdim < 1 || s->dstate < 1)
+        return SSD_ERR_INVALID_ARG;
+    if (s->nheads % s->ngroups != 0) return SSD_ERR_INVALID_ARG;
+    const bool pn_ok = (s->headdim == 64 && s->dstate == 128) || (s->headdim == 16 && s->dstate == 16);
+    if (!pn_ok) return SSD_ERR_UNSUPPORTED;
+    *d = Dims{s->batch, 1, s->nheads, s->headdim, s->ngroups, s->dstate, 1, 1, s->nheads / s->ngroups, 1};
+    return SSD_OK;
+}
+
+ssd_status ssd_decode_step_bf16(const ssd_shape* shape, const uint16_t* x, const float* dt, const float* A,
+                                const uint16_t* B, const uint16_t* C, const float* D, float* state, uint16_t* y,
+                                cudaStream_t stream) {
+    Dims d;
+    const ssd_status st = decode_dims(shape, &d);
+    if (st != SSD_OK) return st;
+    if (!A || !D) return SSD_ERR_INVALID_ARG;
+    if (d.B == 0) return SSD_OK;
+    if (!x || !dt || !B || !C || !state || !y) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dt) || !aligned16(B) || !aligned16(C) || !aligned16(state) || !aligned16(y))
+        return SSD_ERR_INVALID_ARG;
+    SSD_STAGE("decode_step", launch_decode_bf16(d, x, dt, A, B, C, D, state, y, stream));
+    return SSD_OK;
+}
+
+ssd_status ssd_decode_step_i8(const ssd_shape* shape, const uint16_t* x, const float* dt, const float* A,
+                              const int8_t* Bq, const int8_t* Cq, const float* D, const ssd_i8_params* params,
+                              int8_t* state, uint16_t* y, cudaStream_t stream) {
+    Dims d;
+    const ssd_status st = decode_dims(shape, &d);
+    if (st != SSD_OK) return st;
+    if (!A || !D) return SSD_ERR_INVALID_ARG;
+    if (!params || !params->s_B || !params->s_C || !params->s_x || !params->s_s) return SSD_ERR_INVALID_ARG;
+    if (params->decay_shift < 1 || params->decay_shift > 14) return SSD_ERR_INVALID_ARG;
+    if (d.B == 0) return SSD_OK;
+    if (!x || !dt || !Bq || !Cq || !state || !y) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dt) || !aligned16(Bq) || !aligned16(Cq) || !aligned16(state) || !aligned16(y))
+        return SSD_ERR_INVALID_ARG;
+    const I8Scales sc{params->s_B, params->s_C, params->s_x, params->s_s, params->decay_shift};
+    SSD_STAGE("decode_step", launch_decode_i8(d, x, dt, A, Bq, Cq, D, sc, state, y, stream));
+    return SSD_OK;
+}
+
 static WsLayout calib_layout(const Dims& p, size_t* fin_off, size_t* amax_off) {
     WsLayout w = ws_layout(p, false, true);
     *fin_off = w.total;

@@ -197,3 +197,43 @@ class StreamedScan:
                 self.h["y"][r0:r0 + n].copy_(sl["y"][:n], non_blocking=True)
                 self.h["final"][r0:r0 + n].copy_(sl["final"][:n], non_blocking=True)
                 self.ev["out"][k].record(s_out)
+
+
+class Decoder:
+    """One-token steps on a persistent state (serving after a scan).
+
+    state: the scan's final state to continue from — fp32 [B,H,P,N] (bf16 path) or
+    int8 codes [B,H,P,N] (W8A8, real value code * s_s) — updated in place by each step.
+    A, D: device fp32 [H].  W8A8 takes the static scales (device tensors s_B, s_C, s_x, s_s).
+    Each step takes the token's x [B,H,P] (bf16), dt [B,H], B and C [B,G,N] (bf16) and
+    returns y [B,H,P] (bf16, a buffer reused by the next step).
+    """
+
+    def __init__(self, state, A, D, path: str, scales: dict | None = None, shift: int = 7):
+        assert path in ("bf16", "w8a8")
+        self.state, self.A, self.D, self.path = state, A, D, path
+        b, H, P, N = state.shape
+        self.dims = (b, H, P, N)
+        self.y = torch.empty((b, H, P), dtype=torch.bfloat16, device=state.device)
+        self.params = None
+        if path == "w8a8":
+            self.scales = scales
+            self.params = ssd.i8_params(scales["s_B"], scales["s_C"], scales["s_x"], scales["s_s"], shift)
+            self.Bq = self.Cq = None
+
+    def _shape(self, B):
+        b, H, P, N = self.dims
+        return ssd.SsdShape.of(b, 1, H, P, B.shape[-2], N, 256)
+
+    def step(self, x, dt, B, C, stream=None):
+        shape = self._shape(B)
+        if self.path == "bf16":
+            ssd.ssd_decode_step_bf16(shape, x, dt, self.A, B, C, self.D, self.state, self.y, stream)
+            return self.y
+        if self.Bq is None or self.Bq.shape != B.shape:
+            self.Bq = torch.empty(B.shape, dtype=torch.int8, device=B.device)
+            self.Cq = torch.empty(B.shape, dtype=torch.int8, device=B.device)
+        ssd.ssd_quantize_inputs(shape, B, C, self.scales["s_B"], self.scales["s_C"], self.Bq, self.Cq, stream)
+        ssd.ssd_decode_step_i8(shape, x, dt, self.A, self.Bq, self.Cq, self.D, self.params, self.state, self.y,
+                               stream)
+        return self.y

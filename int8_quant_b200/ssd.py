@@ -22,7 +22,8 @@ EXPORTS = ("ssd_status_string", "ssd_last_cuda_error", "ssd_workspace_bytes", "s
            "ssd_scan_fwd_i8", "ssd_scan_fwd_i8_debug", "ssd_calibrate_workspace_bytes",
            "ssd_calibrate_i8", "ssd_workspace_status", "ssd_profile_enable", "ssd_profile_read",
            "ssd_profile_reset", "ssd_scan_fwd_bf16_static", "ssd_selftest_bounded_wait",
-           "ssd_scan_fwd_bf16_from_state", "ssd_scan_fwd_i8_from_state")
+           "ssd_scan_fwd_bf16_from_state", "ssd_scan_fwd_i8_from_state", "ssd_decode_step_bf16",
+           "ssd_decode_step_i8")
 
 # Size of the library's fixed device scratch used by ssd_scan_fwd_bf16_static.
 STATIC_SCRATCH_BYTES = 32 << 20
@@ -87,6 +88,10 @@ def _lib():
         lib.ssd_scan_fwd_i8_from_state.restype = I
         lib.ssd_scan_fwd_i8_from_state.argtypes = [sp, P, P, P, P, P, P, ctypes.POINTER(SsdI8Params), P, P, P, P,
                                                    S, P]
+        lib.ssd_decode_step_bf16.restype = I
+        lib.ssd_decode_step_bf16.argtypes = [sp, P, P, P, P, P, P, P, P, P]
+        lib.ssd_decode_step_i8.restype = I
+        lib.ssd_decode_step_i8.argtypes = [sp, P, P, P, P, P, P, ctypes.POINTER(SsdI8Params), P, P, P]
         lib.ssd_scan_fwd_bf16_static.restype = I
         lib.ssd_scan_fwd_bf16_static.argtypes = [sp, P, P, P, P, P, P, P, P, P]
         lib.ssd_scan_fwd_i8.restype = I
@@ -172,6 +177,18 @@ def ssd_scan_fwd_i8_from_state(shape, x, dt, A, Bq, Cq, D, params: SsdI8Params, 
         ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bq), _ptr(Cq), _ptr(D), ctypes.byref(params),
         _ptr(initial_state), _ptr(y), _ptr(final_state), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def ssd_decode_step_bf16(shape, x, dt, A, B, C, D, state, y, stream=None):
+    _check("ssd_decode_step_bf16", _lib().ssd_decode_step_bf16(
+        ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(state), _ptr(y),
+        _stream(stream)))
+
+
+def ssd_decode_step_i8(shape, x, dt, A, Bq, Cq, D, params: SsdI8Params, state, y, stream=None):
+    _check("ssd_decode_step_i8", _lib().ssd_decode_step_i8(
+        ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bq), _ptr(Cq), _ptr(D), ctypes.byref(params),
+        _ptr(state), _ptr(y), _stream(stream)))
 
 
 def ssd_scan_fwd_bf16_static(shape, x, dt, A, B, C, D, y, final_state, stream=None):

@@ -109,3 +109,20 @@ def test_bounded_wait_selftest_validates_before_any_launch():
     assert lib.ssd_selftest_bounded_wait(1 << 40, f, f, None) == 1      # beyond the kernels' own limit
     assert lib.ssd_selftest_bounded_wait(1000, None, f, None) == 1      # null status
     assert lib.ssd_selftest_bounded_wait(1000, f, None, None) == 1      # null cycles
+
+
+def test_decode_step_validates_before_any_launch():
+    lib = iq.library()
+    f = _fake()
+    one = iq.SsdShape.of(2, 1, 4, 64, 1, 128, 256)
+    two = iq.SsdShape.of(2, 2, 4, 64, 1, 128, 256)                    # seqlen must be 1
+    bad = iq.SsdShape.of(2, 1, 4, 32, 1, 64, 256)                     # unsupported (P, N)
+    assert lib.ssd_decode_step_bf16(ctypes.byref(two), f, f, f, f, f, f, f, f, None) == 1
+    assert lib.ssd_decode_step_bf16(ctypes.byref(bad), f, f, f, f, f, f, f, f, None) == 2
+    assert lib.ssd_decode_step_bf16(ctypes.byref(one), f, f, f, f, f, f, None, f, None) == 1     # null state
+    assert lib.ssd_decode_step_bf16(ctypes.byref(one), f, f, f, f, f, f, f, _fake(0x10004), None) == 1
+    p = iq.SsdI8Params(0x10000, 0x10000, 0x10000, 0x10000, 7)
+    assert lib.ssd_decode_step_i8(ctypes.byref(one), f, f, f, f, f, f, None, f, f, None) == 1    # no params
+    p.decay_shift = 0
+    assert lib.ssd_decode_step_i8(ctypes.byref(one), f, f, f, f, f, f, ctypes.byref(p), f, f, None) == 1
+    assert lib.ssd_decode_step_bf16(None, f, f, f, f, f, f, f, f, None) == 1
