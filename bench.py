@@ -344,6 +344,44 @@ def run_ours(args, rank, world, dist):
                 "peak_source": peak_src,
                 "kernel_shares": {k: round(v[0] / sum(x[0] for x in kern.values()), 4) for k, v in kern.items()}}
 
+    def decode(path, steps=50, warm=5):
+        """One-token steps continuing the scan's final state (ssd_decode_step_*, one launch
+        per token; W8A8 quantises the token's B and C inside).  L2 is refilled with other
+        data before every step (a read of 256 MB, which leaves no dirty lines to write
+        back), so each step reads and writes the whole state from HBM, as it would between
+        the other layers of a model; the time is the decode kernel's own (CUDA events
+        around each launch), not the refill."""
+        from int8_quant_b200.runner import Decoder
+        state = (pb.final8 if path == "w8a8" else pb.final32).clone()
+        dec = Decoder(state, dinp["A"], dinp["D"], path, pb.scales if path == "w8a8" else None)
+        toks = [{k: dinp[k][:, t].contiguous() for k in ("x", "dt", "B", "C")} for t in range(8)]
+        flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        for i in range(warm):
+            dec.step(**toks[i % 8], stream=stream)
+        torch.cuda.synchronize()
+        iq.ssd_profile_reset()
+        for i in range(steps):
+            with torch.cuda.stream(stream):
+                flush.amax()
+            iq.ssd_profile_enable(True)
+            dec.step(**toks[i % 8], stream=stream)
+            iq.ssd_profile_enable(False)
+        torch.cuda.synchronize()
+        kern = iq.ssd_profile_read()
+        us = {k: v[0] / max(v[1], 1) * 1e3 for k, v in kern.items()}
+        step_us = sum(us.values())
+        b, H, P, N, G = w.batch, w.nheads, w.headdim, w.dstate, w.ngroups
+        eb = 1 if path == "w8a8" else 4
+        alg = b * H * P * N * eb * 2 + b * H * P * 4 + b * H * 4 + b * G * N * 4
+        k_us = us.get("decode_step", 0.0)
+        return {"tokens_per_s": round(b / (step_us * 1e-6), 1), "us_per_step": round(step_us, 3),
+                "kernels_us": {k: round(v, 3) for k, v in us.items()},
+                "roofline": {"kernel": "decode_step", "bound": "hbm", "alg_bytes": alg,
+                             "achieved": round(alg / (k_us * 1e-6) / 1e9, 1) if k_us else None, "peak": peak,
+                             "unit": "GB/s", "frac": round(alg / (k_us * 1e-6) / 1e9 / peak, 4) if k_us else None},
+                "state": f"{'int8' if path == 'w8a8' else 'fp32'} [{b},{H},{P},{N}], continuing the scan's final state",
+                "l2": "refilled with 256 MB of other reads before every step"}
+
     def e2e(path):
         """Same metric with the batch in pinned host memory: every step copies the inputs in and y and
         the final state out, group by group (StreamedScan), overlapping the copies with the scans."""
@@ -387,6 +425,8 @@ def run_ours(args, rank, world, dist):
         }
         if not args.no_e2e:
             results[path]["e2e"] = e2e(path)
+    if not args.no_decode:
+        results["decode"] = {p: decode(p) for p in paths}
     return w, results
 
 
@@ -398,6 +438,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2-2.7b", choices=sorted(WORKLOADS))
     ap.add_argument("--path", choices=["w8a8", "bf16"], default="w8a8")
+    ap.add_argument("--no-decode", action="store_true", help="skip the one-token decode-step measurement")
     ap.add_argument("--only-path", action="store_true", help="time only --path (profiling runs)")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")
     ap.add_argument("--seqlen", type=int, default=None, help="override the workload's length (profiling runs)")
@@ -491,6 +532,8 @@ def main():
         "clocks": main_r["clocks"],
         "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in main_r["kern"].items()},
     }
+    if "decode" in res:
+        line["decode"] = res["decode"]
     if o is not None:
         line[other] = {"value": o["value"], "ms_per_step": round(o["ms_per_step"], 5), "roofline": o["roofline"],
                        "path_roofline": o["path_roofline"], "e2e": o.get("e2e"), "gpu_launches": o["gpu_launches"],

@@ -238,16 +238,17 @@ ssd_status ssd_decode_step_bf16(const ssd_shape* shape, const uint16_t* x, const
 
 /* W8A8 one-token step on the INT8 state of ssd_scan_fwd_i8 (codes, real value code *
  * s_s[h*P+p]), in place: the scan's integer steps with a chunk of one token ("SSDi8"
- * notes, key designs 1-2, eq. 6), so that the state codes equal those of
- * ssd_scan_fwd_i8_from_state over that token:
+ * notes, key designs 1-3, eq. 6), so that the state codes equal those of
+ * ssd_quantize_inputs + ssd_scan_fwd_i8_from_state over that token:
+ *   Bq, Cq = the token's B, C quantised as ssd_quantize_inputs does (per group)
  *   a = dt*A;  Xq = clamp(rint(dt*x / s_x));  S8 = clamp(rint((Xq*Bq) * (s_x*s_B/s_s)))
  *   dq = rint(exp(a) * 2^k);  H <- sat127(S8 + ((dq*H + 2^(k-1)) >> k))
  *   y = (Cq.H_before)*s_C*s_s*exp(a) + (Cq.Bq)*s_C*s_B*dt*x + D*x     (bf16)
- * Bq, Cq : device int8 [B, G, N] (ssd_quantize_inputs with seqlen 1).  params as in
- * ssd_scan_fwd_i8.  state : device int8 [B, H, P, N], read and overwritten.  Other
- * arguments as in ssd_decode_step_bf16. */
+ * B, C : device bf16 [B, G, N] (one launch per token: no separate quantisation call).
+ * params as in ssd_scan_fwd_i8.  state : device int8 [B, H, P, N], read and overwritten.
+ * Other arguments as in ssd_decode_step_bf16. */
 ssd_status ssd_decode_step_i8(const ssd_shape* shape, const uint16_t* x, const float* dt, const float* A,
-                              const int8_t* Bq, const int8_t* Cq, const float* D, const ssd_i8_params* params,
+                              const uint16_t* B, const uint16_t* C, const float* D, const ssd_i8_params* params,
                               int8_t* state, uint16_t* y, cudaStream_t stream);
 
 /* Self-test of the device-side bounded wait (the mechanism behind SSD_ERR_TIMEOUT):

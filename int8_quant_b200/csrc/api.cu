@@ -403,7 +403,7 @@ ssd_status ssd_decode_step_bf16(const ssd_shape* shape, const uint16_t* x, const
 }
 
 ssd_status ssd_decode_step_i8(const ssd_shape* shape, const uint16_t* x, const float* dt, const float* A,
-                              const int8_t* Bq, const int8_t* Cq, const float* D, const ssd_i8_params* params,
+                              const uint16_t* B, const uint16_t* C, const float* D, const ssd_i8_params* params,
                               int8_t* state, uint16_t* y, cudaStream_t stream) {
     Dims d;
     const ssd_status st = decode_dims(shape, &d);
@@ -412,11 +412,11 @@ ssd_status ssd_decode_step_i8(const ssd_shape* shape, const uint16_t* x, const f
     if (!params || !params->s_B || !params->s_C || !params->s_x || !params->s_s) return SSD_ERR_INVALID_ARG;
     if (params->decay_shift < 1 || params->decay_shift > 14) return SSD_ERR_INVALID_ARG;
     if (d.B == 0) return SSD_OK;
-    if (!x || !dt || !Bq || !Cq || !state || !y) return SSD_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(dt) || !aligned16(Bq) || !aligned16(Cq) || !aligned16(state) || !aligned16(y))
+    if (!x || !dt || !B || !C || !state || !y) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dt) || !aligned16(B) || !aligned16(C) || !aligned16(state) || !aligned16(y))
         return SSD_ERR_INVALID_ARG;
     const I8Scales sc{params->s_B, params->s_C, params->s_x, params->s_s, params->decay_shift};
-    SSD_STAGE("decode_step", launch_decode_i8(d, x, dt, A, Bq, Cq, D, sc, state, y, stream));
+    SSD_STAGE("decode_step", launch_decode_i8(d, x, dt, A, B, C, D, sc, state, y, stream));
     return SSD_OK;
 }
 

@@ -4,16 +4,18 @@
 //   h <- exp(dt*A) * h + dt * x B^T        y = C . h + D * x
 // bf16 path: fp32 state.  W8A8 path: the INT8 state of the scan (real value code *
 // s_s[h,p]) updated by the scan's own integer steps with a chunk of one token ("SSDi8"
-// notes, key designs 1-2 and eq. 6): the chunk's cumulative sum is a = dt*A, the state
+// notes, key designs 1-3 and eq. 6): the token's B and C are quantised per group as at
+// the scan's entry, the chunk's cumulative sum is a = dt*A, the state
 // LUT is dt * exp(a - a) = dt, X_scaled = dt * x is quantised per (h,p), the INT32
 // product Xq * Bq is requantised to INT8 with s_x*s_B/s_s, and the state carried over
 // the token is (dq * H + 2^(k-1)) >> k with dq = rint(exp(a) * 2^k); y is ChunkScan1
 // (Cq . H on the state before the token, times s_C*s_s*exp(a)) plus ChunkScan2 (the
 // single CB = Cq . Bq, times s_C*s_B*dt, as a bf16 factor of x) plus D*x.
 //
-// Both are one pass over the state (read and write once): one (b,h,p) row of N
-// elements per N/4 lanes, four consecutive elements per lane (a 16-byte fp32 or
-// 4-byte INT8 access), the row's C . h reduced by shuffles.
+// Both are one pass over the state (read and write once), one (b,h,p) row of N
+// elements per group of lanes with a 16-byte access each (four fp32 elements, or
+// sixteen INT8 codes, per lane), the state load issued before anything else; the
+// row's C . h is reduced by shuffles.
 #include "kernels.h"
 
 namespace ssd {
@@ -50,93 +52,150 @@ __global__ void __launch_bounds__(kThreads)
 decode_bf16_kernel(Dims d, const uint16_t* __restrict__ x, const float* __restrict__ dt, const float* __restrict__ A,
                    const uint16_t* __restrict__ Bm, const uint16_t* __restrict__ Cm, const float* __restrict__ D,
                    float* __restrict__ state, uint16_t* __restrict__ y) {
-    constexpr int LPR = N / 4;                                   // lanes per state row
+    constexpr int VPL = N >= 64 ? 2 : 1;                          // float4s per lane (32 bytes in flight)
+    constexpr int LPR = N / (4 * VPL);                            // lanes per state row
     const long long rows = (long long)d.B * d.H * d.P;
     const long long row = ((long long)blockIdx.x * kThreads + threadIdx.x) / LPR;
-    const int sub = threadIdx.x % LPR, n0 = 4 * sub;
+    const int sub = threadIdx.x % LPR;
     const bool active = row < rows;                               // whole lane groups, shuffles stay full-warp
     const RowIdx i = row_of(d, active ? row : 0);
     float part = 0.f, xv = 0.f;
     if (active) {
+        // lane `sub` holds elements [4 (sub + LPR v), +4) for v < VPL: each access a coalesced row slice
+        float4* sp = reinterpret_cast<float4*>(state + i.r * N);
+        float4 h4[VPL];
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) h4[v] = sp[sub + LPR * v];
         const long long bh = (long long)i.b * d.H + i.h;
         const float dtv = __ldg(dt + bh);
         const float dA = expf(dtv * __ldg(A + i.h));
         xv = bf16_bits_to_float(x[i.r]);
         const float u = dtv * xv;
-        const uint2 bw = __ldg(reinterpret_cast<const uint2*>(Bm + ((long long)i.b * d.G + i.g) * N + n0));
-        const uint2 cw = __ldg(reinterpret_cast<const uint2*>(Cm + ((long long)i.b * d.G + i.g) * N + n0));
-        const float bv[4] = {__uint_as_float(bw.x << 16), __uint_as_float(bw.x & 0xffff0000u),
-                             __uint_as_float(bw.y << 16), __uint_as_float(bw.y & 0xffff0000u)};
-        const float cv[4] = {__uint_as_float(cw.x << 16), __uint_as_float(cw.x & 0xffff0000u),
-                             __uint_as_float(cw.y << 16), __uint_as_float(cw.y & 0xffff0000u)};
-        float4* sp = reinterpret_cast<float4*>(state + i.r * N + n0);
-        const float4 h4 = *sp;
-        float hv[4] = {h4.x, h4.y, h4.z, h4.w};
+        const uint2* bp = reinterpret_cast<const uint2*>(Bm + ((long long)i.b * d.G + i.g) * N);
+        const uint2* cp = reinterpret_cast<const uint2*>(Cm + ((long long)i.b * d.G + i.g) * N);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            hv[v] = fmaf(dA, hv[v], u * bv[v]);
-            part = fmaf(cv[v], hv[v], part);
+        for (int v = 0; v < VPL; ++v) {
+            const uint2 bw = __ldg(bp + sub + LPR * v), cw = __ldg(cp + sub + LPR * v);
+            const float bv[4] = {__uint_as_float(bw.x << 16), __uint_as_float(bw.x & 0xffff0000u),
+                                 __uint_as_float(bw.y << 16), __uint_as_float(bw.y & 0xffff0000u)};
+            const float cv[4] = {__uint_as_float(cw.x << 16), __uint_as_float(cw.x & 0xffff0000u),
+                                 __uint_as_float(cw.y << 16), __uint_as_float(cw.y & 0xffff0000u)};
+            float hv[4] = {h4[v].x, h4[v].y, h4[v].z, h4[v].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                hv[e] = fmaf(dA, hv[e], u * bv[e]);
+                part = fmaf(cv[e], hv[e], part);
+            }
+            sp[sub + LPR * v] = make_float4(hv[0], hv[1], hv[2], hv[3]);
         }
-        *sp = make_float4(hv[0], hv[1], hv[2], hv[3]);
     }
     part = row_sum<LPR>(part);
     if (active && sub == 0) y[i.r] = float_to_bf16_bits(fmaf(__ldg(D + i.h), xv, part));
 }
 
-template <int N>
+// Round-to-nearest-even of |v| < 2^22 to an int, and an int of magnitude < 2^22 to
+// float, exactly and without conversion instructions: 1.5 * 2^23 + v is representable
+// with the rounded value in its low mantissa bits (bit pattern 0x4B400000 + value).
+__device__ __forceinline__ int rne_small(float v) { return __float_as_int(__fadd_rn(v, 12582912.0f)) - 0x4B400000; }
+__device__ __forceinline__ float small_to_float(int a) { return __fsub_rn(__int_as_float(a + 0x4B400000), 12582912.0f); }
+// clamp(rint(v * inv), +-127): the clamp first, then the rounding (the same result)
+__device__ __forceinline__ int code_of(float v, float inv) {
+    return rne_small(fminf(fmaxf(__fmul_rn(v, inv), -127.0f), 127.0f));
+}
+
+// RPT state rows of one (b, h) per lane group (rows p, p + RS, ...; RS lane groups per
+// warp): the token's B, C codes and the head's decay are formed once for them, and
+// RPT 16-byte state loads are in flight per lane.
+template <int N, int RPT>
 __global__ void __launch_bounds__(kThreads)
 decode_i8_kernel(Dims d, const uint16_t* __restrict__ x, const float* __restrict__ dt, const float* __restrict__ A,
-                 const int8_t* __restrict__ Bq, const int8_t* __restrict__ Cq, const float* __restrict__ D,
+                 const uint16_t* __restrict__ Bm, const uint16_t* __restrict__ Cm, const float* __restrict__ D,
                  I8Scales sc, int8_t* __restrict__ state, uint16_t* __restrict__ y) {
-    constexpr int LPR = N / 4;
+    constexpr int LPR = N / 16;                                  // lanes per state row, 16 codes each
+    constexpr int RS = 32 / LPR;                                 // lane groups per warp
     const long long rows = (long long)d.B * d.H * d.P;
-    const long long row = ((long long)blockIdx.x * kThreads + threadIdx.x) / LPR;
-    const int sub = threadIdx.x % LPR, n0 = 4 * sub;
-    const bool active = row < rows;
-    const RowIdx i = row_of(d, active ? row : 0);
-    int acc1 = 0, cb = 0;
-    float xv = 0.f, a = 0.f, dtv = 0.f;
-    if (active) {
-        const long long bh = (long long)i.b * d.H + i.h;
-        const int hp = i.h * d.P + i.p;
-        dtv = __ldg(dt + bh);
-        a = __fmul_rn(dtv, __ldg(A + i.h));                        // ChunkCumsum of the one-token chunk
-        xv = bf16_bits_to_float(x[i.r]);
-        // ChunkState: X_scaled = LUT_state * x with LUT_state = dt * exp(a - a), its code
-        const float lut = __fmul_rn(dtv, ssd_expf(__fsub_rn(a, a)));
-        const float sx = __ldg(sc.s_x + hp);
-        const int xq = quant_i8(__fmul_rn(lut, xv), __frcp_rn(sx));
-        const float M = __fdiv_rn(__fmul_rn(sx, __ldg(sc.s_B + i.g)), __ldg(sc.s_s + hp));
-        // StatePassing: the decay code and the rounding shift
-        const int dq = (int)rintf(__fmul_rn(ssd_expf(a), (float)(1 << sc.shift)));
-        const int half = 1 << (sc.shift - 1);
-        const long long gn = ((long long)i.b * d.G + i.g) * N + n0;
-        const uint32_t bw = __ldg(reinterpret_cast<const uint32_t*>(Bq + gn));
-        const uint32_t cw = __ldg(reinterpret_cast<const uint32_t*>(Cq + gn));
-        uint32_t* sp = reinterpret_cast<uint32_t*>(state + i.r * N + n0);
-        const uint32_t hw = *sp;
-        uint32_t out = 0;
+    const long long grp = ((long long)blockIdx.x * kThreads + threadIdx.x) / LPR;
+    const long long row0 = (grp / RS) * (RS * RPT) + grp % RS;  // this group's first row; the others + k RS
+    const int sub = threadIdx.x % LPR, n0 = 16 * sub;
+    const bool active = row0 < rows;                             // a group's rows share (b, h): P % (RS*RPT) == 0
+    const RowIdx i = row_of(d, active ? row0 : 0);
+    int acc1[RPT], cb = 0;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const int hs = (int)(int8_t)(hw >> (8 * v));
-            const int bq = (int)(int8_t)(bw >> (8 * v));
-            const int cq = (int)(int8_t)(cw >> (8 * v));
-            const int s8 = quant_i8((float)(xq * bq), M);          // requantised INT32 state contribution
-            const int hn = sat127(s8 + ((dq * hs + half) >> sc.shift));
-            out |= ((uint32_t)hn & 0xffu) << (8 * v);
-            acc1 += cq * hs;                                      // ChunkScan1 on the state before the token
-            cb += cq * bq;                                        // ChunkBMM of the token with itself
+    for (int k = 0; k < RPT; ++k) acc1[k] = 0;
+    float xv[RPT], a = 0.f, dtv = 0.f;
+    if (active) {
+        uint4* sp = reinterpret_cast<uint4*>(state + i.r * N + n0);
+        uint4 hw4[RPT];
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) hw4[k] = sp[(long long)k * RS * N / 16];
+        const long long gn = ((long long)i.b * d.G + i.g) * N + n0;
+        const uint4* bp = reinterpret_cast<const uint4*>(Bm + gn);          // 16 bf16 = two 16-byte loads
+        const uint4* cp = reinterpret_cast<const uint4*>(Cm + gn);
+        const uint4 braw[2] = {__ldg(bp), __ldg(bp + 1)};
+        const uint4 craw[2] = {__ldg(cp), __ldg(cp + 1)};
+        const long long bh = (long long)i.b * d.H + i.h;
+        dtv = __ldg(dt + bh);
+        const float Ah = __ldg(A + i.h), sB = __ldg(sc.s_B + i.g), sC = __ldg(sc.s_C + i.g);
+        float sx[RPT], ss[RPT];
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const int hp = i.h * d.P + i.p + k * RS;
+            sx[k] = __ldg(sc.s_x + hp);
+            ss[k] = __ldg(sc.s_s + hp);
+            xv[k] = bf16_bits_to_float(x[i.r + k * RS]);
         }
-        *sp = out;
+        a = __fmul_rn(dtv, Ah);                                   // ChunkCumsum of the one-token chunk
+        const float lut = __fmul_rn(dtv, ssd_expf(__fsub_rn(a, a)));   // LUT_state = dt * exp(a - a)
+        const int dq = (int)rintf(__fmul_rn(ssd_expf(a), (float)(1 << sc.shift)));   // decay code
+        const int half = 1 << (sc.shift - 1);
+        // the token's B and C codes, as ssd_quantize_inputs forms them: clamp(rint(v * (1/s)), +-127)
+        const float invB = __frcp_rn(sB), invC = __frcp_rn(sC);
+        const uint32_t bb[8] = {braw[0].x, braw[0].y, braw[0].z, braw[0].w, braw[1].x, braw[1].y, braw[1].z, braw[1].w};
+        const uint32_t cc[8] = {craw[0].x, craw[0].y, craw[0].z, craw[0].w, craw[1].x, craw[1].y, craw[1].z, craw[1].w};
+        int bqv[16], cqv[16];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            bqv[2 * e] = code_of(__uint_as_float(bb[e] << 16), invB);
+            bqv[2 * e + 1] = code_of(__uint_as_float(bb[e] & 0xffff0000u), invB);
+            cqv[2 * e] = code_of(__uint_as_float(cc[e] << 16), invC);
+            cqv[2 * e + 1] = code_of(__uint_as_float(cc[e] & 0xffff0000u), invC);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) cb += cqv[e] * bqv[e];       // ChunkBMM of the token with itself
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            // ChunkState: X_scaled = LUT_state * x, its code; the requantisation factor
+            const int xq = code_of(__fmul_rn(lut, xv[k]), __frcp_rn(sx[k]));
+            const float M = __fdiv_rn(__fmul_rn(sx[k], sB), ss[k]);
+            const uint32_t hw[4] = {hw4[k].x, hw4[k].y, hw4[k].z, hw4[k].w};
+            uint32_t out[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                out[q] = 0;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int hs = (int)(int8_t)(hw[q] >> (8 * v));
+                    const int s8 = code_of(small_to_float(xq * bqv[4 * q + v]), M);   // requantised contribution
+                    const int hn = sat127(s8 + ((dq * hs + half) >> sc.shift));
+                    out[q] |= ((uint32_t)hn & 0xffu) << (8 * v);
+                    acc1[k] += cqv[4 * q + v] * hs;               // ChunkScan1 on the state before the token
+                }
+            }
+            sp[(long long)k * RS * N / 16] = make_uint4(out[0], out[1], out[2], out[3]);
+        }
     }
-    acc1 = row_sum<LPR>(acc1);
     cb = row_sum<LPR>(cb);
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) acc1[k] = row_sum<LPR>(acc1[k]);
     if (active && sub == 0) {
-        const int hp = i.h * d.P + i.p;
         const float sC = __ldg(sc.s_C + i.g);
-        const float y_o = (float)acc1 * (sC * __ldg(sc.s_s + hp)) * expf(a);
         const float m = bf16_bits_to_float(float_to_bf16_bits((float)cb * (sC * __ldg(sc.s_B + i.g)) * dtv));
-        y[i.r] = float_to_bf16_bits(fmaf(__ldg(D + i.h), xv, fmaf(m, xv, y_o)));
+        const float ea = expf(a), Dh = __ldg(D + i.h);
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const float y_o = (float)acc1[k] * (sC * __ldg(sc.s_s + i.h * d.P + i.p + k * RS)) * ea;
+            y[i.r + k * RS] = float_to_bf16_bits(fmaf(Dh, xv[k], fmaf(m, xv[k], y_o)));
+        }
     }
 }
 
@@ -144,7 +203,7 @@ decode_i8_kernel(Dims d, const uint16_t* __restrict__ x, const float* __restrict
 
 cudaError_t launch_decode_bf16(const Dims& d, const uint16_t* x, const float* dt, const float* A, const uint16_t* B,
                                const uint16_t* C, const float* D, float* state, uint16_t* y, cudaStream_t st) {
-    const long long threads = (long long)d.B * d.H * d.P * (d.N / 4);
+    const long long threads = (long long)d.B * d.H * d.P * (d.N >= 64 ? d.N / 8 : d.N / 4);
     if (threads == 0) return cudaSuccess;
     const unsigned grid = (unsigned)((threads + kThreads - 1) / kThreads);
     if (d.N == 128) decode_bf16_kernel<128><<<grid, kThreads, 0, st>>>(d, x, dt, A, B, C, D, state, y);
@@ -153,14 +212,17 @@ cudaError_t launch_decode_bf16(const Dims& d, const uint16_t* x, const float* dt
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode_i8(const Dims& d, const uint16_t* x, const float* dt, const float* A, const int8_t* Bq,
-                             const int8_t* Cq, const float* D, const I8Scales& sc, int8_t* state, uint16_t* y,
+cudaError_t launch_decode_i8(const Dims& d, const uint16_t* x, const float* dt, const float* A, const uint16_t* Bq,
+                             const uint16_t* Cq, const float* D, const I8Scales& sc, int8_t* state, uint16_t* y,
                              cudaStream_t st) {
-    const long long threads = (long long)d.B * d.H * d.P * (d.N / 4);
+    // N = 128 (P = 64): 4 rows per lane group, 16 rows of one head per warp; N = 16: one row
+    constexpr int kRpt128 = 4;
+    if (d.N == 128 && d.P % (4 * kRpt128) != 0) return cudaErrorInvalidValue;
+    const long long threads = (long long)d.B * d.H * d.P * (d.N / 16) / (d.N == 128 ? kRpt128 : 1);
     if (threads == 0) return cudaSuccess;
     const unsigned grid = (unsigned)((threads + kThreads - 1) / kThreads);
-    if (d.N == 128) decode_i8_kernel<128><<<grid, kThreads, 0, st>>>(d, x, dt, A, Bq, Cq, D, sc, state, y);
-    else if (d.N == 16) decode_i8_kernel<16><<<grid, kThreads, 0, st>>>(d, x, dt, A, Bq, Cq, D, sc, state, y);
+    if (d.N == 128) decode_i8_kernel<128, kRpt128><<<grid, kThreads, 0, st>>>(d, x, dt, A, Bq, Cq, D, sc, state, y);
+    else if (d.N == 16) decode_i8_kernel<16, 1><<<grid, kThreads, 0, st>>>(d, x, dt, A, Bq, Cq, D, sc, state, y);
     else return cudaErrorInvalidValue;
     return cudaGetLastError();
 }

@@ -66,11 +66,11 @@ cudaError_t launch_chunk_state_i8(const Dims& d, const uint16_t* x, const float*
 //         chunk as bf16 (Hc) and/or fp32 (Hc32), the final state as fp32.
 //   W8A8: H_{c+1} = sat127(S8_c + ((dq_c * H_c + 2^(k-1)) >> k)).
 // One token on the persistent state (in place): bf16 path on an fp32 state, W8A8 on the
-// INT8 state codes.  x [B,H,P] bf16, dt [B,H], B/C (or Bq/Cq) [B,G,N], y [B,H,P] bf16.
+// INT8 state codes (B and C quantised inside).  x [B,H,P] bf16, dt [B,H], B/C bf16 [B,G,N], y [B,H,P] bf16.
 cudaError_t launch_decode_bf16(const Dims& d, const uint16_t* x, const float* dt, const float* A, const uint16_t* B,
                                const uint16_t* C, const float* D, float* state, uint16_t* y, cudaStream_t st);
-cudaError_t launch_decode_i8(const Dims& d, const uint16_t* x, const float* dt, const float* A, const int8_t* Bq,
-                             const int8_t* Cq, const float* D, const I8Scales& sc, int8_t* state, uint16_t* y,
+cudaError_t launch_decode_i8(const Dims& d, const uint16_t* x, const float* dt, const float* A, const uint16_t* B,
+                             const uint16_t* C, const float* D, const I8Scales& sc, int8_t* state, uint16_t* y,
                              cudaStream_t st);
 
 // init (fp32 [B,H,P,N]) / init8 (INT8 codes [B,H,P,N]): the state before the first chunk, or null for zero.

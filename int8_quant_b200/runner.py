@@ -219,7 +219,6 @@ class Decoder:
         if path == "w8a8":
             self.scales = scales
             self.params = ssd.i8_params(scales["s_B"], scales["s_C"], scales["s_x"], scales["s_s"], shift)
-            self.Bq = self.Cq = None
 
     def _shape(self, B):
         b, H, P, N = self.dims
@@ -230,10 +229,5 @@ class Decoder:
         if self.path == "bf16":
             ssd.ssd_decode_step_bf16(shape, x, dt, self.A, B, C, self.D, self.state, self.y, stream)
             return self.y
-        if self.Bq is None or self.Bq.shape != B.shape:
-            self.Bq = torch.empty(B.shape, dtype=torch.int8, device=B.device)
-            self.Cq = torch.empty(B.shape, dtype=torch.int8, device=B.device)
-        ssd.ssd_quantize_inputs(shape, B, C, self.scales["s_B"], self.scales["s_C"], self.Bq, self.Cq, stream)
-        ssd.ssd_decode_step_i8(shape, x, dt, self.A, self.Bq, self.Cq, self.D, self.params, self.state, self.y,
-                               stream)
+        ssd.ssd_decode_step_i8(shape, x, dt, self.A, B, C, self.D, self.params, self.state, self.y, stream)
         return self.y

@@ -185,9 +185,9 @@ def ssd_decode_step_bf16(shape, x, dt, A, B, C, D, state, y, stream=None):
         _stream(stream)))
 
 
-def ssd_decode_step_i8(shape, x, dt, A, Bq, Cq, D, params: SsdI8Params, state, y, stream=None):
+def ssd_decode_step_i8(shape, x, dt, A, B, C, D, params: SsdI8Params, state, y, stream=None):
     _check("ssd_decode_step_i8", _lib().ssd_decode_step_i8(
-        ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bq), _ptr(Cq), _ptr(D), ctypes.byref(params),
+        ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), ctypes.byref(params),
         _ptr(state), _ptr(y), _stream(stream)))
 
 

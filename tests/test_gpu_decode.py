@@ -103,7 +103,6 @@ def test_i8_decode_steps_bit_exact(torch_cuda, name):
         torch.cuda.synchronize()
         r = W.decode_step_i8(x[:, t], inp["dt"][:, t], inp["A"], Bq[:, t], Cq[:, t], inp["D"], sc["s_B"], sc["s_C"],
                              sc["s_x"], sc["s_s"], ref)
-        np.testing.assert_array_equal(host(dec.Bq), Bq[:, t])
         np.testing.assert_array_equal(host(dec.state), r["state8"])
         assert rel_l2(y, r["y"]) <= 1e-2, (t, rel_l2(y, r["y"]))
         ref = r["state8"]
