@@ -215,8 +215,8 @@ cudaError_t launch_decode_bf16(const Dims& d, const uint16_t* x, const float* dt
 cudaError_t launch_decode_i8(const Dims& d, const uint16_t* x, const float* dt, const float* A, const uint16_t* Bq,
                              const uint16_t* Cq, const float* D, const I8Scales& sc, int8_t* state, uint16_t* y,
                              cudaStream_t st) {
-    // N = 128 (P = 64): 4 rows per lane group, 16 rows of one head per warp; N = 16: one row
-    constexpr int kRpt128 = 4;
+    // N = 128 (P = 64): 2 rows per lane group, 8 rows of one head per warp (measured best of 1, 2, 4); N = 16: one row
+    constexpr int kRpt128 = 2;
     if (d.N == 128 && d.P % (4 * kRpt128) != 0) return cudaErrorInvalidValue;
     const long long threads = (long long)d.B * d.H * d.P * (d.N / 16) / (d.N == 128 ? kRpt128 : 1);
     if (threads == 0) return cudaSuccess;
