@@ -19,6 +19,8 @@ Modules:
   force, fp64 chunked form (ChunkCumsum … ChunkScan); calibration.
 * `ssd_w8a8`  — the integer W8A8 pipeline with its fp32 prelude specified op by
   op, so that every integer it produces is reproducible bit for bit.
+* `study_xscaled` — quantisation error of Q(X_scaled) against Q(X)⊙LUT_state
+  (the comparison of key design 1's appendix claim), measured on given inputs.
 
 Parity status per function is listed in each module's docstring.
 """
