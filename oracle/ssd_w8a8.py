@@ -145,9 +145,17 @@ def state_passing_i8(S8: np.ndarray, dq: np.ndarray, k: int = 7, init8=None) -> 
     return out
 
 
-def ssd_w8a8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, chunk: int, k: int = 7, init8=None) -> dict:
+def ssd_w8a8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, chunk: int, k: int = 7, init8=None,
+             acs_fp16: bool = False, cb_int8: bool = False) -> dict:
     """The W8A8 SSD forward from the INT8 state init8 ([Bt,H,P,N], real value
     init8·s_s; None is the zero state).
+
+    acs_fp16, cb_int8: the notes' storage variant, for the accuracy study only (the
+    library implements neither): dAcs kept in FP16 ("overall framework": dAcs is
+    tiny and stays FP16), i.e. every later use reads Acs rounded to IEEE half; CB
+    requantised to INT8 before ChunkScan2 (key design 2: CB is quantised to save
+    memory), read here as one step per (b, c, g) tile, amax|CB| / 127 (amax 0 gives 1),
+    with rint and ±127 clamping.
 
     x_vals : float32 values of the bf16 x, [Bt,L,H,P]
     dt [Bt,L,H], A [H], D [H] : float32
@@ -193,6 +201,8 @@ def ssd_w8a8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, chunk: int, k: int = 
     a = (dtp * A[None, None, :]).astype(F32)                            # dt·A
     a_h = np.ascontiguousarray(np.moveaxis(a.reshape(Bt, nc, Q, H), 3, 1))   # [Bt,H,nc,Q]
     Acs = chunk_cumsum_f32(a_h)
+    if acs_fp16:
+        Acs = Acs.astype(np.float16).astype(F32)
     last = Acs[..., Q - 1:Q]                                            # [Bt,H,nc,1]
 
     # ChunkState with the decay moved onto x, quantised per (H,P)
@@ -229,7 +239,15 @@ def ssd_w8a8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, chunk: int, k: int = 
     causal = np.tril(np.ones((Q, Q), dtype=bool))
     dec = np.where(causal, np.exp(np.where(causal, diff, 0.0)), 0.0)
     sCB = (s_C.astype(f64) * s_B.astype(f64))[gh]                       # [H]
-    CBh = CB[:, :, gh].astype(f64)                                      # [Bt,nc,H,Q,Q]
+    if cb_int8:
+        amax = np.abs(CB).max(axis=(-2, -1), keepdims=True).astype(f64)
+        s_cb = np.where(amax > 0, amax / QMAX, 1.0)
+        CB8 = np.clip(np.rint(CB / s_cb), -QMAX, QMAX)
+        CBd = CB8 * s_cb                                                # dequantised INT8 CB
+    else:
+        CB8 = s_cb = None
+        CBd = CB.astype(f64)
+    CBh = CBd[:, :, gh]                                                 # [Bt,nc,H,Q,Q]
     lut2 = sCB[None, :, None, None, None] * dec * dt_h.astype(f64)[..., None, :]   # [Bt,H,nc,Q,Q]
     Mmat = CBh * np.moveaxis(lut2, 1, 2)                                # [Bt,nc,H,Q,Q]
     xc = xp.astype(f64).reshape(Bt, nc, Q, H, P)
@@ -246,6 +264,7 @@ def ssd_w8a8(x_vals, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, chunk: int, k: int = 
         "Acs": Acs, "dq": dq, "Xq": Xq, "acc_state": acc_state.astype(np.int32), "S8": S8,
         "H8": H8[:, :nc], "CB": CB.astype(np.int32), "acc_scan1": acc_scan1.astype(np.int32),
         "lut_state": lut_state, "M": M,
+        **({"CB8": CB8.astype(np.int8), "s_cb": s_cb} if cb_int8 else {}),
     }
 
 

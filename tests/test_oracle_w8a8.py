@@ -266,3 +266,40 @@ def test_decode_steps_equal_fp64_exactly_when_representable():
         st = r["state8"]
     assert np.abs(st).max() < 127
     np.testing.assert_allclose(st.astype(np.float64) * s_s.reshape(H, P)[None, :, :, None], fs, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- the notes' storage variant (study switches)
+def test_fp16_acs_is_exact_when_acs_is_representable_in_half():
+    x, dt, A, Bv, Cv, D, s_B, s_C, s_x, s_s, Q = _exact_case(6)
+    A = np.full_like(A, -0.5)                                 # a = -1/16: every Acs is k/16, |Acs| <= 12
+    Bq, Cq = W.quantize_inputs(Bv, Cv, s_B, s_C)
+    r0 = W.ssd_w8a8(x, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, Q)
+    r1 = W.ssd_w8a8(x, dt, A, Bq, Cq, D, s_B, s_C, s_x, s_s, Q, acs_fp16=True)
+    assert np.array_equal(r0["Acs"], r1["Acs"].astype(np.float16).astype(np.float32))
+    for k in ("Xq", "S8", "H8", "final8", "dq", "acc_scan1"):
+        np.testing.assert_array_equal(r0[k], r1[k])
+    np.testing.assert_array_equal(r0["y"], r1["y"])
+
+
+def test_fp16_acs_changes_codes_when_not_representable():
+    w = Workload("t", 1, 512, 4, 8, 16, 1, 256, seed=7)
+    d, x, Bq, Cq, sc = _calibrated(w)
+    kw = dict(A=d["A"], D=d["D"], s_B=sc["s_B"], s_C=sc["s_C"], s_x=sc["s_x"], s_s=sc["s_s"], chunk=256)
+    r0 = W.ssd_w8a8(x, d["dt"], Bq=Bq, Cq=Cq, **kw)
+    r1 = W.ssd_w8a8(x, d["dt"], Bq=Bq, Cq=Cq, acs_fp16=True, **kw)
+    assert not np.array_equal(r0["Acs"], r1["Acs"])
+    assert rel_l2(r1["y"], r0["y"]) < 1e-2
+
+
+def test_int8_cb_is_a_per_tile_symmetric_requantisation():
+    w = Workload("t", 2, 512, 4, 8, 16, 2, 256, seed=8)
+    d, x, Bq, Cq, sc = _calibrated(w)
+    kw = dict(A=d["A"], D=d["D"], s_B=sc["s_B"], s_C=sc["s_C"], s_x=sc["s_x"], s_s=sc["s_s"], chunk=256)
+    r = W.ssd_w8a8(x, d["dt"], Bq=Bq, Cq=Cq, cb_int8=True, **kw)
+    CB, CB8, s = r["CB"].astype(np.float64), r["CB8"].astype(np.float64), r["s_cb"]
+    assert np.all(np.abs(CB8 * s - CB) <= s / 2 + 1e-9)            # rounding to the nearest step
+    assert np.all(np.abs(CB8).max(axis=(-2, -1)) == 127)            # every tile's amax maps to 127
+    r0 = W.ssd_w8a8(x, d["dt"], Bq=Bq, Cq=Cq, **kw)
+    for k in ("Xq", "S8", "H8", "final8", "acc_scan1"):              # only ChunkScan2 reads CB
+        np.testing.assert_array_equal(r0[k], r[k])
+    assert rel_l2(r["y"], r0["y"]) < 1e-2
