@@ -81,6 +81,15 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
 
 
+def measured_bf16_tflops() -> float:
+    """Burst bf16 dense GEMM throughput measured on this machine (TFLOP/s), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f).get("bf16_tflops", 1590.0))
+    return 1590.0
+
+
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
 # capture, keyed by kernel name, with the sha1 of the kernel source it was taken on.
 # A kernel whose source changed since reports null.
@@ -299,6 +308,7 @@ def run_ours(args, rank, world, dist):
         pb.calibrate(w.calib_prefix)            # static W8A8 scales on the prefix (GPU)
     torch.cuda.synchronize()
     peak, peak_src = measured_peaks()
+    bf16_peak = measured_bf16_tflops()
 
     def step_fn(path):
         if path == "w8a8":
@@ -382,6 +392,48 @@ def run_ours(args, rank, world, dist):
                 "state": f"{'int8' if path == 'w8a8' else 'fp32'} [{b},{H},{P},{N}], continuing the scan's final state",
                 "l2": "refilled with 256 MB of other reads before every step"}
 
+    def out_proj(steps=10, warm=3):
+        """The SSD epilogue on the scan's y seen as [B*L, H*P]: RMSNorm codes + the INT8 output
+        projection to d_model = H*P/2 (the 2.7B layer's 2560) on synthetic weights (seeded; the
+        weight codes and the static scales are set up with torch outside the timed region).
+        y (671 MB) is larger than L2, so every launch reads it from HBM."""
+        T, K = w.tokens, w.nheads * w.headdim
+        Dm = K // 2
+        g = torch.Generator(device=dev).manual_seed(0)
+        Wf = torch.randn((Dm, K), generator=g, device=dev) / K ** 0.5
+        s_w = (Wf.abs().amax(dim=1) / 127).contiguous()
+        Wq = torch.clamp(torch.round(Wf / s_w[:, None]), -127, 127).to(torch.int8).contiguous()
+        corr = (1e-3 * torch.randn(Dm, generator=g, device=dev)).contiguous()
+        y2 = pb.y.view(T, K)
+        u = y2[: 4096].float()
+        s_a = float((u * torch.rsqrt(u.pow(2).mean(dim=1, keepdim=True) + 1e-5)).abs().amax() / 127)
+        out = torch.empty((T, Dm), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(iq.ssd_out_proj_workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+        for _ in range(warm):
+            iq.ssd_out_proj_i8(y2, s_a, Wq, s_w, corr, out, ws, stream=stream)
+        torch.cuda.synchronize()
+        iq.ssd_profile_reset()
+        iq.ssd_profile_enable(True)
+        for _ in range(steps):
+            iq.ssd_out_proj_i8(y2, s_a, Wq, s_w, corr, out, ws, stream=stream)
+        iq.ssd_profile_enable(False)
+        torch.cuda.synchronize()
+        assert iq.ssd_out_proj_status(ws, T, K) == 0
+        kern = {k: v[0] / max(v[1], 1) for k, v in iq.ssd_profile_read().items() if v[1]}
+        gemm_ms, norm_ms = kern.get("out_proj_gemm", 0.0), kern.get("out_proj_norm", 0.0)
+        ops = 2.0 * T * K * Dm
+        i8_peak = 2.0 * bf16_peak
+        norm_bytes = T * K * 2 + T * K                     # y read (its second pass per token hits L2), codes written
+        return {"tokens": T, "d_inner": K, "d_model": Dm, "ms_per_call": round(gemm_ms + norm_ms, 5),
+                "tokens_per_s": round(T / ((gemm_ms + norm_ms) * 1e-3), 1),
+                "gemm": {"ms": round(gemm_ms, 5), "bound": "tensor", "achieved": round(ops / (gemm_ms * 1e-3) / 1e12, 1),
+                         "peak": round(i8_peak, 1), "unit": "TOP/s", "frac": round(ops / (gemm_ms * 1e-3) / 1e12 / i8_peak, 4),
+                         "peak_source": "2 x measured bf16 burst (MEASURED_PEAKS.json), the nominal int8/bf16 ratio"},
+                "norm": {"ms": round(norm_ms, 5), "bound": "hbm", "alg_bytes": norm_bytes,
+                         "achieved": round(norm_bytes / (norm_ms * 1e-3) / 1e9, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(norm_bytes / (norm_ms * 1e-3) / 1e9 / peak, 4)},
+                "weights": "synthetic, seeded; corr = synthetic mean-correction vector"}
+
     def e2e(path):
         """Same metric with the batch in pinned host memory: every step copies the inputs in and y and
         the final state out, group by group (StreamedScan), overlapping the copies with the scans."""
@@ -427,6 +479,8 @@ def run_ours(args, rank, world, dist):
             results[path]["e2e"] = e2e(path)
     if not args.no_decode:
         results["decode"] = {p: decode(p) for p in paths}
+    if not args.no_out_proj:
+        results["out_proj"] = out_proj()
     return w, results
 
 
@@ -439,6 +493,7 @@ def main():
     ap.add_argument("--workload", default="mamba2-2.7b", choices=sorted(WORKLOADS))
     ap.add_argument("--path", choices=["w8a8", "bf16"], default="w8a8")
     ap.add_argument("--no-decode", action="store_true", help="skip the one-token decode-step measurement")
+    ap.add_argument("--no-out-proj", action="store_true", help="skip the SSD-epilogue (INT8 out projection) measurement")
     ap.add_argument("--only-path", action="store_true", help="time only --path (profiling runs)")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")
     ap.add_argument("--seqlen", type=int, default=None, help="override the workload's length (profiling runs)")
@@ -534,6 +589,8 @@ def main():
     }
     if "decode" in res:
         line["decode"] = res["decode"]
+    if "out_proj" in res:
+        line["out_proj"] = res["out_proj"]
     if o is not None:
         line[other] = {"value": o["value"], "ms_per_step": round(o["ms_per_step"], 5), "roofline": o["roofline"],
                        "path_roofline": o["path_roofline"], "e2e": o.get("e2e"), "gpu_launches": o["gpu_launches"],

@@ -251,6 +251,30 @@ ssd_status ssd_decode_step_i8(const ssd_shape* shape, const uint16_t* x, const f
                               const uint16_t* B, const uint16_t* C, const float* D, const ssd_i8_params* params,
                               int8_t* state, uint16_t* y, cudaStream_t stream);
 
+/* SSD epilogue of the W8A8 pipeline ("SSDi8" notes, key design 4 and the training
+ * strategy): RMSNorm of the scan output, static symmetric INT8 codes, the output
+ * projection as an INT8 GEMM on the tensor cores, dequantisation and the mean
+ * correction:
+ *   u = y / sqrt(mean_k y^2 + 1e-5)             (per token, over k < d_inner)
+ *   Aq = clamp(rint(u / s_a), +-127)             (codes kept in the workspace)
+ *   out[t,d] = s_a * s_w[d] * sum_k Aq[t,k] Wq[d,k] + corr[d]     (bf16)
+ * The RMSNorm weight is folded into Wq (gamma migration); corr = 0.15 c*, the mean
+ * correction from calibration (null: none).
+ * y : device bf16 [tokens, d_inner] (the scan's y seen as [B*L, H*P])
+ * Wq : device int8 [d_model, d_inner]; s_w, corr : device fp32 [d_model]; s_a > 0
+ * out : device bf16 [tokens, d_model], written
+ * acc_debug : device int32 [tokens, d_model] or null: the INT32 accumulators
+ * workspace : device, at least ssd_out_proj_workspace_bytes(tokens, d_inner) bytes
+ * Supported: d_inner % 128 == 0, d_model % 256 == 0, tokens % 128 == 0 (else
+ * SSD_ERR_UNSUPPORTED).  All pointers 16-byte aligned.  Asynchronous; a device-side
+ * timeout is read back with ssd_out_proj_status. */
+size_t ssd_out_proj_workspace_bytes(int tokens, int d_inner);
+ssd_status ssd_out_proj_i8(int tokens, int d_inner, int d_model, const uint16_t* y, float s_a, const int8_t* Wq,
+                           const float* s_w, const float* corr, uint16_t* out, int32_t* acc_debug, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream);
+/* Synchronises `stream` and returns the status word of an ssd_out_proj_i8 workspace. */
+ssd_status ssd_out_proj_status(void* workspace, int tokens, int d_inner, cudaStream_t stream);
+
 /* Self-test of the device-side bounded wait (the mechanism behind SSD_ERR_TIMEOUT):
  * launches, on `stream`, one CTA of two warps that wait on mbarriers nothing ever
  * completes.  Warp 0 gives up after `limit_cycles` SM clock cycles (0 < limit_cycles

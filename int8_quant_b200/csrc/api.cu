@@ -375,6 +375,40 @@ ssd_status ssd_scan_fwd_i8_from_state(const ssd_shape* shape, const uint16_t* x,
                    nullptr, stream);
 }
 
+size_t ssd_out_proj_workspace_bytes(int tokens, int d_inner) {
+    if (tokens < 0 || d_inner < 1) return 0;
+    return align256((size_t)tokens * d_inner) + 256;
+}
+
+ssd_status ssd_out_proj_i8(int tokens, int d_inner, int d_model, const uint16_t* y, float s_a, const int8_t* Wq,
+                           const float* s_w, const float* corr, uint16_t* out, int32_t* acc_debug, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream) {
+    if (tokens < 0 || d_inner < 1 || d_model < 1 || !(s_a > 0.f)) return SSD_ERR_INVALID_ARG;
+    if (d_inner % 128 != 0 || d_model % 256 != 0 || tokens % 128 != 0) return SSD_ERR_UNSUPPORTED;
+    if (!Wq || !s_w || !aligned16(Wq) || (corr && !aligned16(corr))) return SSD_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < ssd_out_proj_workspace_bytes(tokens, d_inner))
+        return SSD_ERR_WORKSPACE;
+    int* status = at<int>(workspace, align256((size_t)tokens * d_inner));
+    SSD_TRY(cudaMemsetAsync(status, 0, sizeof(int), stream));
+    if (tokens == 0) return SSD_OK;
+    if (!y || !out || !aligned16(y) || !aligned16(out) || (acc_debug && !aligned16(acc_debug)))
+        return SSD_ERR_INVALID_ARG;
+    int8_t* aq = static_cast<int8_t*>(workspace);
+    SSD_STAGE("out_proj_norm", launch_out_proj_norm(tokens, d_inner, y, s_a, aq, stream));
+    SSD_STAGE("out_proj_gemm", launch_out_proj_gemm(tokens, d_inner, d_model, aq, s_a, Wq, s_w, corr, out, acc_debug,
+                                                    status, stream));
+    return SSD_OK;
+}
+
+ssd_status ssd_out_proj_status(void* workspace, int tokens, int d_inner, cudaStream_t stream) {
+    if (!workspace || tokens < 0 || d_inner < 1) return SSD_ERR_INVALID_ARG;
+    int v = 0;
+    SSD_TRY(cudaMemcpyAsync(&v, at<int>(workspace, align256((size_t)tokens * d_inner)), sizeof(int),
+                            cudaMemcpyDeviceToHost, stream));
+    SSD_TRY(cudaStreamSynchronize(stream));
+    return v == 0 ? SSD_OK : (ssd_status)v;
+}
+
 // Shape of a one-token step: seqlen must be 1; chunk is not used.
 static ssd_status decode_dims(const ssd_shape* s, Dims* d) {
     if (!s) return SSD_ERR_INVALID_ARG;

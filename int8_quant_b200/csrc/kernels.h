@@ -73,6 +73,12 @@ cudaError_t launch_decode_i8(const Dims& d, const uint16_t* x, const float* dt, 
                              const uint16_t* C, const float* D, const I8Scales& sc, int8_t* state, uint16_t* y,
                              cudaStream_t st);
 
+// SSD epilogue: RMSNorm codes of y [T,K] (bf16) into aq [T,K], then out [T,D] (bf16) =
+// (aq Wq^T) * s_a * s_w[d] + corr[d] (corr may be null); acc_dbg [T,D] int32 optional.
+cudaError_t launch_out_proj_norm(int T, int K, const uint16_t* y, float s_a, int8_t* aq, cudaStream_t st);
+cudaError_t launch_out_proj_gemm(int T, int K, int D, const int8_t* aq, float s_a, const int8_t* Wq, const float* s_w,
+                                 const float* corr, uint16_t* out, int32_t* acc_dbg, int* status, cudaStream_t st);
+
 // init (fp32 [B,H,P,N]) / init8 (INT8 codes [B,H,P,N]): the state before the first chunk, or null for zero.
 cudaError_t launch_state_passing_bf16(const Dims& d, const void* S, bool s_fp32, const float* decay,
                                       const float* init, uint16_t* Hc, float* final_state, float* amax_h,

@@ -23,7 +23,7 @@ EXPORTS = ("ssd_status_string", "ssd_last_cuda_error", "ssd_workspace_bytes", "s
            "ssd_calibrate_i8", "ssd_workspace_status", "ssd_profile_enable", "ssd_profile_read",
            "ssd_profile_reset", "ssd_scan_fwd_bf16_static", "ssd_selftest_bounded_wait",
            "ssd_scan_fwd_bf16_from_state", "ssd_scan_fwd_i8_from_state", "ssd_decode_step_bf16",
-           "ssd_decode_step_i8")
+           "ssd_decode_step_i8", "ssd_out_proj_workspace_bytes", "ssd_out_proj_i8", "ssd_out_proj_status")
 
 # Size of the library's fixed device scratch used by ssd_scan_fwd_bf16_static.
 STATIC_SCRATCH_BYTES = 32 << 20
@@ -92,6 +92,12 @@ def _lib():
         lib.ssd_decode_step_bf16.argtypes = [sp, P, P, P, P, P, P, P, P, P]
         lib.ssd_decode_step_i8.restype = I
         lib.ssd_decode_step_i8.argtypes = [sp, P, P, P, P, P, P, ctypes.POINTER(SsdI8Params), P, P, P]
+        lib.ssd_out_proj_workspace_bytes.restype = S
+        lib.ssd_out_proj_workspace_bytes.argtypes = [I, I]
+        lib.ssd_out_proj_i8.restype = I
+        lib.ssd_out_proj_i8.argtypes = [I, I, I, P, ctypes.c_float, P, P, P, P, P, P, S, P]
+        lib.ssd_out_proj_status.restype = I
+        lib.ssd_out_proj_status.argtypes = [P, I, I, P]
         lib.ssd_scan_fwd_bf16_static.restype = I
         lib.ssd_scan_fwd_bf16_static.argtypes = [sp, P, P, P, P, P, P, P, P, P]
         lib.ssd_scan_fwd_i8.restype = I
@@ -189,6 +195,23 @@ def ssd_decode_step_i8(shape, x, dt, A, B, C, D, params: SsdI8Params, state, y, 
     _check("ssd_decode_step_i8", _lib().ssd_decode_step_i8(
         ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), ctypes.byref(params),
         _ptr(state), _ptr(y), _stream(stream)))
+
+
+def ssd_out_proj_workspace_bytes(tokens: int, d_inner: int) -> int:
+    return int(_lib().ssd_out_proj_workspace_bytes(int(tokens), int(d_inner)))
+
+
+def ssd_out_proj_i8(y, s_a: float, Wq, s_w, corr, out, workspace, acc_debug=None, stream=None):
+    """y [T, K] bf16; Wq [D, K] int8; s_w, corr [D] fp32 (corr may be None); out [T, D] bf16."""
+    T, K = y.shape
+    D = Wq.shape[0]
+    _check("ssd_out_proj_i8", _lib().ssd_out_proj_i8(
+        T, K, D, _ptr(y), float(s_a), _ptr(Wq), _ptr(s_w), _ptr(corr), _ptr(out), _ptr(acc_debug), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def ssd_out_proj_status(workspace, tokens: int, d_inner: int, stream=None) -> int:
+    return int(_lib().ssd_out_proj_status(_ptr(workspace), int(tokens), int(d_inner), _stream(stream)))
 
 
 def ssd_scan_fwd_bf16_static(shape, x, dt, A, B, C, D, y, final_state, stream=None):

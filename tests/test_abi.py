@@ -126,3 +126,19 @@ def test_decode_step_validates_before_any_launch():
     p.decay_shift = 0
     assert lib.ssd_decode_step_i8(ctypes.byref(one), f, f, f, f, f, f, ctypes.byref(p), f, f, None) == 1
     assert lib.ssd_decode_step_bf16(None, f, f, f, f, f, f, f, f, None) == 1
+
+
+def test_out_proj_validates_before_any_launch():
+    lib = iq.library()
+    f = _fake()
+    ws = lib.ssd_out_proj_workspace_bytes(256, 512)
+    assert ws >= 256 * 512
+    assert lib.ssd_out_proj_workspace_bytes(-1, 512) == 0
+    # unsupported sizes
+    assert lib.ssd_out_proj_i8(256, 500, 512, f, 0.1, f, f, None, f, None, f, ws, None) == 2
+    assert lib.ssd_out_proj_i8(256, 512, 500, f, 0.1, f, f, None, f, None, f, ws, None) == 2
+    assert lib.ssd_out_proj_i8(200, 512, 512, f, 0.1, f, f, None, f, None, f, ws, None) == 2
+    # bad scale, null weights, small workspace
+    assert lib.ssd_out_proj_i8(256, 512, 512, f, 0.0, f, f, None, f, None, f, ws, None) == 1
+    assert lib.ssd_out_proj_i8(256, 512, 512, f, 0.1, None, f, None, f, None, f, ws, None) == 1
+    assert lib.ssd_out_proj_i8(256, 512, 512, f, 0.1, f, f, None, f, None, f, ws - 1, None) == 3
