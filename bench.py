@@ -179,6 +179,12 @@ class ClockSampler:
                 self.source = "nvidia-smi, 100 ms"
             except (OSError, FileNotFoundError):
                 self.proc = None
+                if getattr(self, "fh", None):
+                    self.fh.close()
+                    try:
+                        os.remove(self.path)
+                    except OSError:
+                        pass
         return self
 
     def __exit__(self, *a):
