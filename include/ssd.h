@@ -37,8 +37,14 @@
  *    return SSD_ERR_UNSUPPORTED.
  *  - Preconditions not checked (the values are not scanned): dt >= 0 and finite,
  *    A <= 0, scales > 0 and finite.
- *  - The initial state is zero.
+ *  - The initial state is zero, except in the *_from_state entry points, which take
+ *    one (the format of final_state).
  *  - No C++ exception crosses this interface.
+ *
+ * Beyond the scan, on the same conventions: the one-token decode step on the
+ * persistent state (ssd_decode_step_bf16 / _i8), the SSD epilogue of the W8A8
+ * pipeline (RMSNorm + INT8 output projection with the mean correction,
+ * ssd_out_proj_i8) and a self-test of the device-side bounded wait.
  */
 #ifndef SSD_B200_H
 #define SSD_B200_H
