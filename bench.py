@@ -69,6 +69,8 @@ def kernel_bytes(w, path: str, kernel: str) -> int:
         return states * st_w + chains * nc * 4 + states * hc_w + fin
     if kernel == "chunk_scan":                                  # x, B, C, Acs, dt, passed states in; y out
         return T * (2 * H * P + 2 * bc * G * N + 2 * H * P) + 2 * vec + states * hc_w
+    if kernel == "ssd_fused_i8":                                # the whole scan: x, Bq, Cq, dt in; y, final out
+        return T * (2 * H * P + 2 * G * N + 4 * H + 2 * H * P) + fin + 4 * (2 * G + 2 * H * P) + 8 * H
     return 0
 
 

@@ -1,5 +1,6 @@
 // api.cu — the C ABI of libssd.so: argument validation, workspace layout and the
 // launch sequence of each entry point on the caller's stream.
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -42,6 +43,15 @@ ssd_status make_dims(const ssd_shape* s, Dims* d) {
 // Shapes served by the tensor-core kernels; the (16,16) test shape uses the
 // CUDA-core kernels.
 bool tensor_core_shape(const Dims& d) { return d.P == 64 && d.N == 128; }
+
+// The W8A8 scan of the tensor-core shapes runs as the five-launch sequence (quantize,
+// ChunkCumsum, ChunkState, StatePassing, ChunkScan), the faster of the two designs on
+// B200; SSD_I8_FUSED=1 in the environment selects the single persistent kernel
+// (fused_i8.cu), which gives the same integers bit for bit.
+bool i8_fused(const Dims& d) {
+    const char* e = getenv("SSD_I8_FUSED");
+    return tensor_core_shape(d) && e && e[0] == '1';
+}
 
 }  // namespace
 
@@ -120,6 +130,13 @@ WsLayout ws_layout(const Dims& d, bool i8, bool fp32_states) {
     w.scales = off;  off += align256(i8 ? (size_t)2 * d.H * d.P * sizeof(float) : 0);   // 1/s_x, s_x s_B / s_s
     w.total = off;
     return w;
+}
+
+size_t ws_bytes(const Dims& d, bool i8) {
+    const size_t staged = ws_layout(d, i8).total;
+    if (!i8 || !tensor_core_shape(d)) return staged;
+    const size_t fused = fused_i8_ws_bytes(d);
+    return fused > staged ? fused : staged;
 }
 
 // ---------------------------------------------------------------- per-kernel timing
@@ -202,7 +219,7 @@ const char* ssd_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_er
 size_t ssd_workspace_bytes(const ssd_shape* shape, int is_i8) {
     Dims d;
     if (make_dims(shape, &d) != SSD_OK) return 0;
-    return ws_layout(d, is_i8 != 0).total;
+    return ws_bytes(d, is_i8 != 0);
 }
 
 ssd_status ssd_quantize_inputs(const ssd_shape* shape, const uint16_t* B, const uint16_t* C,
@@ -221,7 +238,7 @@ ssd_status ssd_quantize_inputs(const ssd_shape* shape, const uint16_t* B, const 
 
 static ssd_status check_common(const Dims& d, const void* x, const float* dt, const float* A,
                                const void* B, const void* C, const float* D, const void* y,
-                               const void* final_state, void* ws, size_t ws_bytes, bool i8) {
+                               const void* final_state, void* ws, size_t ws_size, bool i8) {
     if (!final_state || !A || !D) return SSD_ERR_INVALID_ARG;
     if (!aligned16(final_state)) return SSD_ERR_INVALID_ARG;
     if ((long long)d.B * d.L > 0) {
@@ -230,7 +247,7 @@ static ssd_status check_common(const Dims& d, const void* x, const float* dt, co
             return SSD_ERR_INVALID_ARG;
     }
     if (!ws || !aligned16(ws)) return SSD_ERR_WORKSPACE;
-    if (ws_bytes < ws_layout(d, i8).total) return SSD_ERR_WORKSPACE;
+    if (ws_size < ws_bytes(d, i8)) return SSD_ERR_WORKSPACE;
     return SSD_OK;
 }
 
@@ -315,13 +332,18 @@ static ssd_status scan_i8(const ssd_shape* shape, const uint16_t* x, const float
             return from_cuda(cudaMemcpyAsync(final_state, initial_state, fs_bytes, cudaMemcpyDeviceToDevice, stream));
         return from_cuda(cudaMemsetAsync(final_state, 0, fs_bytes, stream));
     }
+    I8Scales sc{params->s_B, params->s_C, params->s_x, params->s_s, params->decay_shift};
+    I8Debug dd{};
+    if (dbg) dd = I8Debug{dbg->Acs, dbg->dq, dbg->Xq, dbg->acc_state, dbg->S8, dbg->H8, dbg->cb, dbg->acc_scan1};
+    if (i8_fused(d)) {
+        SSD_STAGE("ssd_fused_i8", launch_fused_i8(d, x, dt, A, Bq, Cq, D, sc, initial_state, y, final_state, workspace,
+                                                  dbg ? &dd : nullptr, stream));
+        return SSD_OK;
+    }
     float* Acs = at<float>(workspace, w.acs);
     int32_t* dq = at<int32_t>(workspace, w.decay);
     int8_t* S8 = at<int8_t>(workspace, w.states);
     int8_t* H8 = at<int8_t>(workspace, w.passed);
-    I8Scales sc{params->s_B, params->s_C, params->s_x, params->s_s, params->decay_shift};
-    I8Debug dd{};
-    if (dbg) dd = I8Debug{dbg->Acs, dbg->dq, dbg->Xq, dbg->acc_state, dbg->S8, dbg->H8, dbg->cb, dbg->acc_scan1};
     float* lut = at<float>(workspace, w.lut);
     float* dtc = at<float>(workspace, w.dtc);
     int* status = at<int>(workspace, w.status);

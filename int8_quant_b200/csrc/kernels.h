@@ -123,6 +123,37 @@ cudaError_t launch_chunk_state_tc(const Dims& d, bool i8, const uint16_t* x, con
                                   const float* lut, const float* inv_sx, const float* mq, uint16_t* S, int8_t* S8,
                                   const I8Debug* dbg, int* status, cudaStream_t st);
 
+// The whole W8A8 scan of one call (ChunkCumsum .. epilogue) as one persistent kernel
+// for P = 64, N = 128 (fused_i8.cu).  Arguments of the kernel:
+struct FusedI8Args {
+    Dims d;
+    int K;            // heads per work item
+    int nhb_g;        // head blocks per group
+    int nhb;          // head blocks per (batch row, chunk)
+    int items;        // B * nc * nhb work items, chunk-major
+    const float* dt;
+    const float* A;
+    const float* D;
+    I8Scales sc;
+    int* status;      // device status word (SSD_ERR_TIMEOUT on an expired wait)
+    int* ticket;      // work-item counter, zero at launch
+    int* hflag;       // [B, nc, H]: quarters of the state entering the chunk published (4 = ready)
+    int8_t* Hpub;     // [B, nc, H, N, P] state entering each chunk (transposed)
+    const float* inv_sx;  // [H*P] 1/s_x
+    const float* mq;      // [H*P] s_x s_B / s_s (requantisation multiplier)
+    const float* mulC;    // [H*P] s_C s_s (ChunkScan1 dequantisation)
+    const int8_t* init8;
+    int8_t* final8;
+    I8Debug dbg;
+};
+// Workspace bytes of the fused W8A8 scan; *ctrl_bytes receives the size of the leading
+// region (status word, ticket, flags) that is cleared before every launch.
+size_t fused_i8_ws_bytes(const Dims& d, size_t* ctrl_bytes = nullptr);
+int fused_heads_per_item(const Dims& d);
+cudaError_t launch_fused_i8(const Dims& d, const uint16_t* x, const float* dt, const float* A, const int8_t* Bq,
+                            const int8_t* Cq, const float* D, const I8Scales& sc, const int8_t* init8, uint16_t* y,
+                            int8_t* final8, void* ws, const I8Debug* dbg, cudaStream_t st);
+
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 // SSD_OK for cudaSuccess; otherwise SSD_ERR_CUDA, remembering `e` for ssd_last_cuda_error.
