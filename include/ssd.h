@@ -135,16 +135,26 @@ ssd_status ssd_scan_fwd_bf16(const ssd_shape* shape, const uint16_t* x, const fl
  *    process exits.  A shape whose ssd_workspace_bytes(shape, 0) exceeds it is
  *    rejected with SSD_ERR_WORKSPACE before anything is enqueued.
  *  - Nothing is allocated: no cudaMalloc/cudaFree or allocating library routine.
- *  - The first call on each device looks up the array's device address (once per
- *    device, with that device current); make that first call before any stream
- *    capture.
+ *  - Every call looks up the array's device address with the calling device current
+ *    (so a cudaDeviceReset or another context never sees a stale address).  Under lazy
+ *    module loading (the CUDA default) the first call on a device loads the library's
+ *    module, and the driver reserves the array's memory then: make that first call at
+ *    start-up, before an arena takes the device's memory and before any stream capture.
  *  - All calls share the one array, which keeps the last call's contents (each call
  *    rewrites what it reads).  Calls whose GPU work overlaps (other streams, other
- *    host threads) race on it: serialise them. */
+ *    host threads) race on it: serialise them.
+ *  - A device-side error of the call (SSD_ERR_TIMEOUT from a bounded wait) is recorded
+ *    in the array's status word: read it with ssd_static_scratch_status. */
 ssd_status ssd_scan_fwd_bf16_static(const ssd_shape* shape, const uint16_t* x, const float* dt,
                                     const float* A, const uint16_t* B, const uint16_t* C,
                                     const float* D, uint16_t* y, float* final_state,
                                     cudaStream_t stream);
+
+/* Status word of the fixed scratch used by ssd_scan_fwd_bf16_static (the counterpart of
+ * ssd_workspace_status for callers that own no workspace): synchronises `stream`, returns
+ * SSD_OK or the error a kernel of the last static call recorded (e.g. SSD_ERR_TIMEOUT),
+ * and clears it.  Allocates nothing. */
+ssd_status ssd_static_scratch_status(cudaStream_t stream);
 
 /* ssd_scan_fwd_bf16 continuing from a given state: h_{-1} = initial_state (device fp32
  * [B, H, P, N], 16-byte aligned; null means zero, as in ssd_scan_fwd_bf16).  Feeding

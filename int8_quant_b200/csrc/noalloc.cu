@@ -9,8 +9,6 @@
 // the status word) in a fixed array in the library's own device memory, sized at
 // compile time.  Every GPU that loads the library holds that array until the
 // process exits, so it is kept modest: SSD_STATIC_SCRATCH_BYTES (32 MiB).
-#include <mutex>
-
 #include "../../include/ssd.h"
 #include "kernels.h"
 
@@ -18,23 +16,16 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_scratch[SSD_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_static_scratch on the current device, looked up once per
-// device.  In host code the symbol name is only a host-side handle, so the address
-// the kernels need must come from cudaGetSymbolAddress with that device current.
+// Device address of g_static_scratch in the current device's current context.  In host
+// code the symbol name is only a host-side handle, so the address the kernels need must
+// come from cudaGetSymbolAddress with that device current.  It is looked up on every
+// call (cheap once the module is loaded), so that no cached address can outlive a
+// cudaDeviceReset or belong to another context.  Under lazy module loading the first
+// lookup on a device loads the module and with it the array.
 ssd_status scratch_for_current_device(void** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SSD_ERR_CUDA;
-    std::lock_guard<std::mutex> g(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return SSD_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return SSD_ERR_CUDA;
+    *out = p;
     return SSD_OK;
 }
 
@@ -59,4 +50,19 @@ extern "C" ssd_status ssd_scan_fwd_bf16_static(const ssd_shape* shape, const uin
     // are never seen.
     return ssd_scan_fwd_bf16(shape, x, dt, A, B, C, D, y, final_state, scratch,
                              (size_t)SSD_STATIC_SCRATCH_BYTES, stream);
+}
+
+extern "C" ssd_status ssd_static_scratch_status(cudaStream_t stream) {
+    // the first int of the scratch is the status word that the scan's kernels set
+    void* p = nullptr;
+    const ssd_status st = scratch_for_current_device(&p);
+    if (st != SSD_OK) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return SSD_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SSD_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SSD_ERR_CUDA;
+    }
+    return v == 0 ? SSD_OK : (ssd_status)v;
 }

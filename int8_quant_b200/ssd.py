@@ -23,7 +23,8 @@ EXPORTS = ("ssd_status_string", "ssd_last_cuda_error", "ssd_workspace_bytes", "s
            "ssd_calibrate_i8", "ssd_workspace_status", "ssd_profile_enable", "ssd_profile_read",
            "ssd_profile_reset", "ssd_scan_fwd_bf16_static", "ssd_selftest_bounded_wait",
            "ssd_scan_fwd_bf16_from_state", "ssd_scan_fwd_i8_from_state", "ssd_decode_step_bf16",
-           "ssd_decode_step_i8", "ssd_out_proj_workspace_bytes", "ssd_out_proj_i8", "ssd_out_proj_status")
+           "ssd_decode_step_i8", "ssd_out_proj_workspace_bytes", "ssd_out_proj_i8", "ssd_out_proj_status",
+           "ssd_static_scratch_status")
 
 # Size of the library's fixed device scratch used by ssd_scan_fwd_bf16_static.
 STATIC_SCRATCH_BYTES = 32 << 20
@@ -100,6 +101,8 @@ def _lib():
         lib.ssd_out_proj_status.argtypes = [P, I, I, P]
         lib.ssd_scan_fwd_bf16_static.restype = I
         lib.ssd_scan_fwd_bf16_static.argtypes = [sp, P, P, P, P, P, P, P, P, P]
+        lib.ssd_static_scratch_status.restype = I
+        lib.ssd_static_scratch_status.argtypes = [P]
         lib.ssd_scan_fwd_i8.restype = I
         lib.ssd_scan_fwd_i8.argtypes = [sp, P, P, P, P, P, P, ctypes.POINTER(SsdI8Params), P, P, P, S, P]
         lib.ssd_scan_fwd_i8_debug.restype = I
@@ -221,6 +224,12 @@ def ssd_scan_fwd_bf16_static(shape, x, dt, A, B, C, D, y, final_state, stream=No
     _check("ssd_scan_fwd_bf16_static", _lib().ssd_scan_fwd_bf16_static(
         ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y), _ptr(final_state),
         _stream(stream)))
+
+
+def ssd_static_scratch_status(stream=None) -> int:
+    """Status word of the fixed scratch after the last ssd_scan_fwd_bf16_static call
+    (synchronises the stream, returns 0 or the recorded error, clears it)."""
+    return int(_lib().ssd_static_scratch_status(_stream(stream)))
 
 
 def i8_params(s_B, s_C, s_x, s_s, decay_shift=7) -> SsdI8Params:
