@@ -11,9 +11,11 @@ counter-based) and recomputes them on the host:
   accumulators, ChunkBMM accumulators of the chain's group, final INT8 state),
   y within 1e-2 of the integer oracle's dequantised y and within 5e-2 of fp64;
 * the library's GPU calibration agrees with the oracle's within 1e-4.
-The 64K and 256K long-context sweeps take minutes of input generation; they run
-when SSD_FULLSIZE_LONG=1.
+The long-context sweeps (B = 1, L = 64K and 256K: 256 and 1024 chunks through
+StatePassing) run by default; their inputs take a minute or two to generate, once per
+workload for both paths.  SSD_FULLSIZE_LONG=0 leaves them out.
 """
+import functools
 import os
 
 import numpy as np
@@ -26,7 +28,7 @@ from tests.gpu_common import (TOL_BF16, TOL_I8_Y, bf16_to_np, host, chain_oracle
 
 pytestmark = pytest.mark.gpu
 
-LONG = os.environ.get("SSD_FULLSIZE_LONG", "0") == "1"
+LONG = os.environ.get("SSD_FULLSIZE_LONG", "1") == "1"
 BF16_WORKLOADS = ["mamba2-1.3b", "mamba2-2.7b", "long-16k"] + (["long-64k", "long-256k"] if LONG else [])
 I8_WORKLOADS = ["mamba2-2.7b", "mamba2-8b", "long-16k"] + (["long-64k", "long-256k"] if LONG else [])
 
@@ -48,9 +50,15 @@ def cuda():
     return torch
 
 
+@functools.lru_cache(maxsize=None)
+def _inputs(name):
+    """Host inputs of a workload, generated once for both paths."""
+    return make_inputs(WORKLOADS[name])
+
+
 def _run(cuda, w, i8: bool, scales=None, debug=False):
     from int8_quant_b200.runner import SsdProblem, to_device
-    pb = SsdProblem(to_device(make_inputs(w)), w.chunk, with_i8=i8, with_bf16=not i8)
+    pb = SsdProblem(to_device(_inputs(w.name)), w.chunk, with_i8=i8, with_bf16=not i8)
     dbg = None
     if not i8:
         pb.run_bf16()

@@ -22,6 +22,8 @@ CASES = {
     "tiny-ragged": Workload("tiny-ragged", 3, 77, 8, 16, 16, 2, 64, seed=3),
     "L1": Workload("L1", 2, 1, 4, 64, 128, 1, 256, seed=4),
     "L63": Workload("L63", 1, 63, 4, 16, 16, 1, 64, seed=5),
+    # 20 heads: the tensor-core ChunkScan takes them in blocks of 8, 8 and 4
+    "ragged-heads": Workload("ragged-heads", 1, 512, 20, 64, 128, 1, 256, seed=6),
 }
 
 

@@ -259,3 +259,29 @@ def test_A_zero_with_initial_state_closed_form():
     h = h0[:, None] + np.cumsum(inject, axis=1)                           # h_t = h0 + Σ_{s≤t} dt x Bᵀ
     ey = np.einsum("blhpn,blhn->blhp", h, C[:, :, g]) + D[None, None, :, None] * x
     assert rel_l2(y, ey) < 1e-12 and rel_l2(fin, h[:, -1]) < 1e-12
+
+
+def test_calibrate_state_scale_counts_the_passed_states():
+    """s_s must take the amax over the passed states too: with A = 0 every chunk adds
+    S_c = Q * dt * x * B = 1, so H_c = c and the final state is nc = 4 while every S_c is
+    1 -> s_s = 4/127 (dropping the passed states would give 1/127, dropping the final one
+    3/127); s_x = amax |dt x| / 127 = (1/32)/127 in closed form."""
+    Q, nc = 32, 4
+    L = Q * nc
+    x = np.ones((1, L, 1, 1))
+    dt = np.full((1, L, 1), 1.0 / Q)
+    A = np.zeros(1)
+    B = np.ones((1, L, 1, 1))
+    C = np.ones((1, L, 1, 1))
+    sc = F.calibrate(x, dt, A, B, C, chunk=Q, prefix=L)
+    assert sc["s_s"][0] == np.float32(4.0 / 127)
+    assert sc["s_x"][0] == np.float32((1.0 / Q) / 127)
+    # a single large chunk state that decays away: the amax is that S_c itself
+    x2 = np.zeros((1, L, 1, 1))
+    x2[:, Q:2 * Q] = -3.0                                   # chunk 1 only
+    A2 = np.array([-64.0])                                  # dt*A = -2 per token: decays to ~0 in a chunk
+    sc2 = F.calibrate(x2, dt, A2, B, C, chunk=Q, prefix=L)
+    _, _, parts = F.ssd_chunked(x2, dt, A2, B, C, np.zeros(1), Q, states_only=True)
+    s1 = abs(parts["S"][0, 1].max()) if abs(parts["S"][0, 1].max()) > abs(parts["S"][0, 1].min()) else abs(parts["S"][0, 1].min())
+    assert sc2["s_s"][0] == np.float32(s1 / 127)
+    assert np.abs(parts["H"]).max() <= s1 + 1e-12
