@@ -39,12 +39,24 @@ FALLBACK_HBM_GBS = 6650.0           # used only when MEASURED_PEAKS.json is abse
 
 # ---------------------------------------------------------------- byte counts
 def path_bytes(w, path: str) -> int:
-    """Compulsory bytes of one step: every input read once, every output written once."""
+    """Compulsory bytes of one step: every input read once, every output written once.
+    Per token x 2HP + y 2HP + dt 4H, and B, C at 4GN (bf16) on the bf16 path, 2GN (their
+    INT8 codes) on the W8A8 path; plus the final state, fp32 or INT8."""
     T, H, P, N, G = w.tokens, w.nheads, w.headdim, w.dstate, w.ngroups
-    per_tok = 2 * H * P + 2 * H * P + 4 * G * N + 4 * H      # x, y, B and C (bf16), dt
+    bc = 2 if path == "w8a8" else 4
+    per_tok = 2 * H * P + 2 * H * P + bc * G * N + 4 * H
     fin = w.batch * H * P * N * (4 if path == "bf16" else 1)
-    params = 8 * H + (0 if path == "bf16" else 4 * (2 * G + 2 * H * P))
-    return T * per_tok + fin + params
+    return T * per_tok + fin
+
+
+def config_of(w, path: str, world: int) -> dict:
+    """The workload as both arms print it."""
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
+            "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
+            "path": path, "step": ("ssd_quantize_inputs + ssd_scan_fwd_i8" if path == "w8a8"
+                                   else "ssd_scan_fwd_bf16"),
+            "l2": f"inputs larger than L2 ({path_bytes(w, path) / 1e9:.2f} GB per step), no flush",
+            "parallelism": f"replicas x{world}"}
 
 
 def kernel_bytes(w, path: str, kernel: str) -> int:
@@ -74,6 +86,43 @@ def kernel_bytes(w, path: str, kernel: str) -> int:
     return 0
 
 
+def io_bytes(w, path: str, kernel: str) -> int:
+    """Algorithmic bytes of one launch as the roofline counts them: only the path's own inputs
+    and outputs that the launch reads or writes, each once (no intermediates: chunk states,
+    passed states, per-chunk vectors)."""
+    T, H, P, N, G = w.tokens, w.nheads, w.headdim, w.dstate, w.ngroups
+    bc = 1 if path == "w8a8" else 2                             # bytes per B/C element the scan reads
+    fin = w.batch * H * P * N * (4 if path == "bf16" else 1)
+    if kernel == "quantize_inputs":                             # B, C in (bf16); Bq, Cq out
+        return T * G * N * (2 * 2 + 2 * 1)
+    if kernel == "chunk_cumsum":                                # dt in
+        return T * H * 4
+    if kernel == "chunk_state":                                 # x, B in
+        return T * (2 * H * P + bc * G * N)
+    if kernel == "state_passing":                               # final state out
+        return fin
+    if kernel == "chunk_scan":                                  # x, B, C, dt in; y out
+        return T * (4 * H * P + 2 * bc * G * N + 4 * H)
+    if kernel == "ssd_fused_i8":                                # the whole scan
+        return T * (4 * H * P + 2 * G * N + 4 * H) + fin
+    return 0
+
+
+def path_flops(w, path: str):
+    """Algorithmic (triangular where causal) contraction counts of one step, 2 per MAC:
+    (bf16 FLOPs, INT8 ops).  Per (b, c, h): ChunkState and ChunkScan1 2 Q P N each,
+    ChunkScan2 Q (Q + 1) P; per (b, c, g): ChunkBMM Q (Q + 1) N."""
+    Q, P, N = w.chunk, w.headdim, w.dstate
+    bch = w.batch * w.nchunks * w.nheads
+    bcg = w.batch * w.nchunks * w.ngroups
+    state = scan1 = 2.0 * Q * P * N * bch
+    scan2 = float(Q) * (Q + 1) * P * bch
+    bmm = float(Q) * (Q + 1) * N * bcg
+    if path == "w8a8":
+        return scan2, state + scan1 + bmm
+    return state + scan1 + scan2 + bmm, 0.0
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -96,8 +145,7 @@ def measured_bf16_tflops() -> float:
 # capture, keyed by kernel name, with the sha1 of the kernel source it was taken on.
 # A kernel whose source changed since reports null.
 NCU_TRAFFIC = {
-    # batch-2 capture scaled x4 to the batch-8 launch (traffic grows with the batch);
-    # see profiles/chunk_scan_tc_mamba2-2.7b-b2.md
+    # batch-2 capture scaled x4 to the batch-8 launch (traffic grows with the batch)
     ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.510976e6 + 131.441664e6),
                                             "src_sha1": "d4289772c1f95756fab8af3deacde1b311a52d75"},
     ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (270.597632e6 + 133.411328e6),
@@ -300,6 +348,11 @@ def replica_throughput(tokens_per_rank: int, ms_per_step: float, world: int) -> 
     return world * tokens_per_rank / (ms_per_step / 1e3)
 
 
+def tc_shape(w) -> bool:
+    """(P, N) = (64, 128): the shape the tensor-core kernels (and the single-launch scan) take."""
+    return (w.headdim, w.dstate) == (64, 128)
+
+
 def run_ours(args, rank, world, dist):
     import torch
     import int8_quant_b200 as iq
@@ -318,7 +371,7 @@ def run_ours(args, rank, world, dist):
     peak, peak_src = measured_peaks()
     bf16_peak = measured_bf16_tflops()
 
-    def step_fn(path):
+    def step_fn(path, pb):
         if path == "w8a8":
             return lambda: pb.run_i8(stream)
         return lambda: pb.run_bf16(stream)
@@ -327,8 +380,8 @@ def run_ours(args, rank, world, dist):
         if dist is not None:
             dist.barrier()
 
-    def timed(path):
-        step = step_fn(path)
+    def timed(path, pb=pb):
+        step = step_fn(path, pb)
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize()
@@ -349,18 +402,39 @@ def run_ours(args, rank, world, dist):
         kern = iq.ssd_profile_read()
         return ms, kern, clk.summary()
 
-    def roofline(path, kern):
-        # dominant kernel = largest share of the step's device time
+    def roofline(path, kern, w=w):
+        # dominant kernel = largest share of the step's device time; its algorithmic bytes are
+        # the path inputs and outputs it touches (no intermediates)
         name = max(kern, key=lambda k: kern[k][0])
         tot_ms, calls = kern[name]
         per_launch_s = tot_ms / calls / 1e3
-        alg = kernel_bytes(w, path, name)
+        alg = io_bytes(w, path, name)
         achieved = alg / per_launch_s / 1e9
+        kb = kernel_bytes(w, path, name)
         return {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_for(name, path, w.name),
-                "alg_bytes_per_launch": alg, "launch_ms": round(per_launch_s * 1e3, 4),
-                "peak_source": peak_src,
+                "frac": round(achieved / peak, 4), "frac_of_8TBs": round(achieved / DATASHEET_HBM_GBS, 4),
+                "traffic": traffic_for(name, path, w.name), "alg_bytes_per_launch": alg,
+                "alg_bytes_def": "path inputs and outputs the launch touches, each once",
+                "launch_ms": round(per_launch_s * 1e3, 4), "peak_source": peak_src,
+                "with_intermediates": {"bytes_per_launch": kb, "frac": round(kb / per_launch_s / 1e9 / peak, 4)},
                 "kernel_shares": {k: round(v[0] / sum(x[0] for x in kern.values()), 4) for k, v in kern.items()}}
+
+    def path_roofline(path, ms, w=w):
+        """The step against the benchmark spec's roofline: the slower of the compulsory HBM bytes over
+        8 TB/s and the contractions at the datasheet tensor peaks (bf16 2.25 PFLOP/s, int8
+        4.5 POP/s), and the same with this machine's measured peaks (copy bandwidth; bf16 GEMM,
+        int8 taken as twice it)."""
+        alg = path_bytes(w, path)
+        fb, oi = path_flops(w, path)
+        t = ms / 1e3
+        t_hbm, t_mma = alg / (DATASHEET_HBM_GBS * 1e9), fb / 2.25e15 + oi / 4.5e15
+        t_hbm_m, t_mma_m = alg / (peak * 1e9), fb / (bf16_peak * 1e12) + oi / (2 * bf16_peak * 1e12)
+        return {"alg_bytes": alg, "bf16_flops": fb, "int8_ops": oi, "achieved_GBs": round(alg / t / 1e9, 1),
+                "t_roof_us": round(max(t_hbm, t_mma) * 1e6, 2), "bound": "hbm" if t_hbm >= t_mma else "tensor",
+                "frac": round(max(t_hbm, t_mma) / t, 4),
+                "frac_of_measured": round(max(t_hbm_m, t_mma_m) / t, 4),
+                "frac_of_measured_hbm": round(alg / t / 1e9 / peak, 4),
+                "frac_of_8TBs": round(alg / t / 1e9 / DATASHEET_HBM_GBS, 4)}
 
     def decode(path, steps=50, warm=5):
         """One-token steps continuing the scan's final state (ssd_decode_step_*, one launch
@@ -453,7 +527,7 @@ def run_ours(args, rank, world, dist):
         host_io["final"] = torch.empty_like(fin, device="cpu").pin_memory()
         runner = StreamedScan(host_io, dinp["A"], dinp["D"], w.chunk, path, rows_per_group=1,
                               scales=pb.scales if path == "w8a8" else None, device=dev)
-        n = max(1, min(args.steps, args.e2e_steps))
+        n = max(1, args.steps)
         runner.run()                                             # warm-up
         torch.cuda.synchronize()
         barrier()
@@ -470,25 +544,70 @@ def run_ours(args, rank, world, dist):
                 "ms_per_step": round(ms, 4), "steps": n, "rows_per_group": 1,
                 "api": "ssd_quantize_inputs + ssd_scan_fwd_i8" if path == "w8a8" else "ssd_scan_fwd_bf16"}
 
+    def fused_i8(w=w, pb=pb):
+        """The W8A8 step with the scan as one persistent launch (SSD_I8_FUSED=1): same integers,
+        timed the same way."""
+        old = os.environ.get("SSD_I8_FUSED")
+        os.environ["SSD_I8_FUSED"] = "1"
+        try:
+            ms, kern, clocks = timed("w8a8", pb)
+        finally:
+            if old is None:
+                del os.environ["SSD_I8_FUSED"]
+            else:
+                os.environ["SSD_I8_FUSED"] = old
+        return {"value": replica_throughput(w.tokens, ms, world), "ms_per_step": round(ms, 5),
+                "roofline": roofline("w8a8", kern, w), "path_roofline": path_roofline("w8a8", ms, w),
+                "gpu_launches": sum(c for _, c in kern.values()), "clocks": clocks,
+                "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in kern.items()}}
+
+    def other_config(name):
+        """Device-timed step of another workload on both paths (its own inputs, calibrated the
+        same way); no e2e, decode or epilogue."""
+        wo = WORKLOADS[name]
+        with torch.cuda.stream(stream):
+            di = to_device(make_inputs(wo), dev)
+            po = SsdProblem(di, wo.chunk, with_i8=True, with_bf16=True)
+            po.calibrate(wo.calib_prefix)
+        torch.cuda.synchronize()
+        cfg = config_of(wo, "bf16", world)
+        cfg.update(path="bf16 and w8a8", step="as in the main line, per path",
+                   l2=f"inputs larger than L2 ({path_bytes(wo, 'w8a8') / 1e9:.2f} GB or more per step), no flush")
+        out = {"config": cfg}
+        for path in ("bf16", "w8a8"):
+            ms, kern, clocks = timed(path, po)
+            rf = roofline(path, kern, wo)
+            out[path] = {"value": replica_throughput(wo.tokens, ms, world), "ms_per_step": round(ms, 5),
+                         "path_roofline": path_roofline(path, ms, wo),
+                         "roofline": {k: rf[k] for k in ("kernel", "achieved", "frac", "frac_of_8TBs", "launch_ms")},
+                         "gpu_launches": sum(c for _, c in kern.values()), "clocks": clocks,
+                         "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in kern.items()}}
+        if tc_shape(wo):
+            out["w8a8_fused"] = {k: v for k, v in fused_i8(wo, po).items() if k != "kernels_ms_per_step"}
+        del po, di
+        torch.cuda.empty_cache()
+        return out
+
     results = {}
     paths = (args.path,) if args.only_path else (args.path, "bf16" if args.path == "w8a8" else "w8a8")
     for path in paths:
         ms, kern, clocks = timed(path)
         launches = sum(c for _, c in kern.values())
-        alg = path_bytes(w, path)
         results[path] = {
             "ms_per_step": ms, "value": replica_throughput(w.tokens, ms, world), "kern": kern, "clocks": clocks,
             "roofline": roofline(path, kern), "gpu_launches": launches,
-            "path_roofline": {"alg_bytes": alg, "achieved_GBs": round(alg / (ms / 1e3) / 1e9, 1),
-                              "frac_of_measured_hbm": round(alg / (ms / 1e3) / 1e9 / peak, 4),
-                              "frac_of_8TBs": round(alg / (ms / 1e3) / 1e9 / DATASHEET_HBM_GBS, 4)},
+            "path_roofline": path_roofline(path, ms),
         }
         if not args.no_e2e:
             results[path]["e2e"] = e2e(path)
+    if "w8a8" in paths and tc_shape(w) and not args.no_fused:
+        results["w8a8_fused"] = fused_i8()
     if not args.no_decode:
         results["decode"] = {p: decode(p) for p in paths}
     if not args.no_out_proj:
         results["out_proj"] = out_proj()
+    if args.all_configs:                          # "tiny" is a parity case (launch-bound), not timed
+        results["configs"] = {n: other_config(n) for n in sorted(WORKLOADS) if n not in (w.name, "tiny")}
     return w, results
 
 
@@ -506,7 +625,9 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")
     ap.add_argument("--seqlen", type=int, default=None, help="override the workload's length (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-fused", action="store_true", help="skip the single-launch W8A8 scan measurement")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="also time every other workload on both paths (device time only; adds minutes)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work per CPU worker")
     args = ap.parse_args()
@@ -540,9 +661,9 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.tokens / value,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64" if args.path == "bf16" else "int64", "data": "synthetic",
-                "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
-                           "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
-                           "path": args.path},
+                "config": config_of(w, args.path, args.gpus),
+                "ms_per_step_note": ("extrapolated: the workload's B*L tokens over the oracle's throughput "
+                                     "on sampled chains, not a timed whole step"),
                 "cpu_baseline": {"kind": "oracle", "cores": vals[0]["cores"], "sample": vals[0]["sample"],
                                  "value": value, "unit": "tokens/s"},
                 "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -584,17 +705,16 @@ def main():
         "warmup": args.warmup, "ms_per_step": round(main_r["ms_per_step"], 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8" if args.path == "w8a8" else "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
-                   "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
-                   "path": args.path, "step": ("ssd_quantize_inputs + ssd_scan_fwd_i8" if args.path == "w8a8"
-                                               else "ssd_scan_fwd_bf16"),
-                   "l2": f"inputs larger than L2 ({path_bytes(w, args.path) / 1e9:.2f} GB per step), no flush",
-                   "parallelism": f"replicas x{world}"},
+        "config": config_of(w, args.path, world),
         "roofline": main_r["roofline"], "path_roofline": main_r["path_roofline"],
         "cpu_baseline": cpu, "e2e": main_r.get("e2e"), "gpu_launches": main_r["gpu_launches"],
         "clocks": main_r["clocks"],
         "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in main_r["kern"].items()},
     }
+    if "w8a8_fused" in res:
+        line["w8a8_fused"] = res["w8a8_fused"]
+    if "configs" in res:
+        line["configs"] = res["configs"]
     if "decode" in res:
         line["decode"] = res["decode"]
     if "out_proj" in res:

@@ -193,7 +193,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + K::OFF_TMEM);
     const long long vec_row0 = (((long long)b * d.H) * d.nc + c) * Q;   // + h * nc * Q
     const long long hc_row0 = ((long long)b * d.nc + c) * d.H;           // state rows (hc_row0 + h) * 64
-    const float sCB = kI8 ? __ldg(sc.s_C + g) * __ldg(sc.s_B + g) : 1.f;
+    const float sCB = kI8 ? __fmul_rn(__ldg(sc.s_C + g), __ldg(sc.s_B + g)) : 1.f;
 
     if (tid == 0) {
         for (int i = 0; i < K::NBAR; ++i) {
@@ -572,13 +572,14 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     vec(s, kMul)[p] = __ldg(sc.s_C + g) * __ldg(sc.s_s + h * kP + p);
                 }
                 for (int i = tid - kScaleWarp0 * 32; i < Q; i += kEpiThreads) {
-                    const float ai = acs[i] * kLog2e;
-                    const float ar = acs[i | 31] * kLog2e;
-                    const float dw = dts[i] * sCB;
+                    // explicitly rounded steps (no contraction), as in the single-launch scan
+                    const float ai = __fmul_rn(acs[i], kLog2e);
+                    const float ar = __fmul_rn(acs[i | 31], kLog2e);
+                    const float dw = __fmul_rn(dts[i], sCB);
                     a2[i] = ai;
-                    dtw[i] = lg2(dw) - ai;                        // log2(dt_i) - a_i; -inf when dt_i = 0
+                    dtw[i] = __fsub_rn(lg2(dw), ai);              // log2(dt_i) - a_i; -inf when dt_i = 0
                     // column factors as bf16 pairs (consecutive lanes hold consecutive i)
-                    const float vi = ex2(fminf(ar - ai, 0.f)) * dw;
+                    const float vi = __fmul_rn(ex2(fminf(__fsub_rn(ar, ai), 0.f)), dw);
                     const float vn = __shfl_down_sync(0xffffffffu, vi, 1);
                     if ((i & 1) == 0) reinterpret_cast<uint32_t*>(v32)[i / 2] = pack_bf16(vi, vn);
                 }
@@ -592,7 +593,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             const uint32_t ybase = trow + K::YCOL + 128 * s;
             for (int J = 0; J < K::JT; ++J) {
                 const int j = J * 128 + r;
-                const float e = ex2(fminf(acs[j < Q ? j : Q - 1] * kLog2e, 0.f));
+                const float e = ex2(fminf(__fmul_rn(acs[j < Q ? j : Q - 1], kLog2e), 0.f));
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     uint32_t v[32];

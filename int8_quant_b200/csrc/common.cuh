@@ -66,6 +66,18 @@ __device__ __forceinline__ int quant_i8(float v, float inv_scale) {
 
 __device__ __forceinline__ int sat127(int v) { return v < -127 ? -127 : (v > 127 ? 127 : v); }
 
+// Lane-wise unsigned min / max of two 16-bit fields per word.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // atomicMax on non-negative floats through their (monotone) bit patterns.
 __device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
     atomicMax(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));

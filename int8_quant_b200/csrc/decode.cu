@@ -199,6 +199,146 @@ decode_i8_kernel(Dims d, const uint16_t* __restrict__ x, const float* __restrict
     }
 }
 
+// (P, N) = (64, 128): one (b, h) per CTA of 128 threads.  The token's B and C codes,
+// the head's decay code and each row's X_scaled code and requantisation factor are
+// formed once per CTA, into shared memory, while the state loads are in flight; then
+// each lane carries 4 rows x 16 codes (rows rb, rb + 16, ...; 8 lanes per row): the
+// requantised contribution on fp32 pairs, ChunkScan1 and ChunkBMM by dp4a, and for
+// decay shifts k <= 7 (and dq <= 2^k) the eq. 6 carry on two codes per 32-bit word: with
+// Hu = H + 128 and Su = S8 + 128, V = dq Hu + 2^(k-1) + 128 (2^k - dq) + Su 2^k
+// = dq H + 2^(k-1) + (S8 + 256) 2^k < 2^16, V >> k = H' + 256 before saturation, so
+// clamping V to [129 2^k, 384 2^k - 1] saturates and the low byte of V >> k is H'.
+constexpr int kHeadThreads = 128;
+
+__global__ void __launch_bounds__(kHeadThreads)
+decode_i8_head_kernel(Dims d, const uint16_t* __restrict__ x, const float* __restrict__ dt,
+                      const float* __restrict__ A, const uint16_t* __restrict__ Bm, const uint16_t* __restrict__ Cm,
+                      const float* __restrict__ D, I8Scales sc, int8_t* __restrict__ state, uint16_t* __restrict__ y) {
+    constexpr int P = 64, N = 128, RPT = 4;
+    __shared__ __align__(16) float s_bqf[N];
+    __shared__ __align__(16) int8_t s_bq[N];
+    __shared__ __align__(16) int8_t s_cq[N];
+    __shared__ float s_xqf[P], s_M[P], s_ys[P], s_xv[P];
+    __shared__ int s_dq;
+    __shared__ float s_ea;
+    const int t = threadIdx.x, sub = t & 7, rb = t >> 3;
+    const long long bh = blockIdx.x;
+    const int b = (int)(bh / d.H), h = (int)(bh % d.H), g = h / d.hpg;
+    uint4* sp = reinterpret_cast<uint4*>(state + bh * (P * N)) + sub;      // row p at sp[p * N / 16]
+    uint4 hw4[RPT];
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) hw4[j] = sp[(rb + 16 * j) * (N / 16)];
+    const float dtv = __ldg(dt + bh);
+    const float a = __fmul_rn(dtv, __ldg(A + h));                   // ChunkCumsum of the one-token chunk
+    const float sB = __ldg(sc.s_B + g), sC = __ldg(sc.s_C + g);
+    if (t < P) {
+        // row p: X_scaled = LUT_state * x with LUT_state = dt * exp(a - a), its code; the
+        // requantisation factor s_x s_B / s_s; y's factor s_C s_s
+        const int p = t, hp = h * P + p;
+        const float sx = __ldg(sc.s_x + hp), ss = __ldg(sc.s_s + hp);
+        const float lut = __fmul_rn(dtv, ssd_expf(__fsub_rn(a, a)));
+        const float xv = bf16_bits_to_float(x[bh * P + p]);
+        s_xv[p] = xv;
+        s_xqf[p] = (float)code_of(__fmul_rn(lut, xv), __frcp_rn(sx));
+        s_M[p] = __fdiv_rn(__fmul_rn(sx, sB), ss);
+        s_ys[p] = sC * ss;
+    } else {
+        // the token's B and C codes n and n + 64, as ssd_quantize_inputs forms them
+        const int n = t - P;
+        const long long gn = ((long long)b * d.G + g) * N;
+        const float invB = __frcp_rn(sB), invC = __frcp_rn(sC);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int nn = n + 64 * e;
+            const int bq = code_of(bf16_bits_to_float(Bm[gn + nn]), invB);
+            s_bqf[nn] = (float)bq;
+            s_bq[nn] = (int8_t)bq;
+            s_cq[nn] = (int8_t)code_of(bf16_bits_to_float(Cm[gn + nn]), invC);
+        }
+        if (n == 0) s_dq = (int)rintf(__fmul_rn(ssd_expf(a), (float)(1 << sc.shift)));   // decay code
+        if (n == 1) s_ea = expf(a);
+    }
+    __syncthreads();
+    const uint4 bq4 = *reinterpret_cast<const uint4*>(s_bq + 16 * sub);
+    const uint4 cq4 = *reinterpret_cast<const uint4*>(s_cq + 16 * sub);
+    const int bw[4] = {(int)bq4.x, (int)bq4.y, (int)bq4.z, (int)bq4.w};
+    const int cw[4] = {(int)cq4.x, (int)cq4.y, (int)cq4.z, (int)cq4.w};
+    int cb = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) cb = __dp4a(cw[q], bw[q], cb);           // ChunkBMM of the token with itself
+    cb = row_sum<8>(cb);
+    float2 bqf[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 f = *reinterpret_cast<const float4*>(s_bqf + 16 * sub + 4 * q);
+        bqf[2 * q] = make_float2(f.x, f.y);
+        bqf[2 * q + 1] = make_float2(f.z, f.w);
+    }
+    const int k = sc.shift, dq = s_dq;
+    const bool packed = k <= 7 && dq <= (1 << k);                          // dq <= 2^k when A dt <= 0
+    const uint32_t k0 = (uint32_t)((1 << (k - 1)) + 128 * ((1 << k) - dq));
+    const uint32_t k0x2 = k0 | (k0 << 16);
+    const uint32_t lo = (129u << k) * 0x10001u, hi = ((384u << k) - 1u) * 0x10001u;
+    const float2 lim_lo = make_float2(-127.0f, -127.0f), lim_hi = make_float2(127.0f, 127.0f);
+    const float2 rnd = make_float2(12582912.0f + 128.0f, 12582912.0f + 128.0f);   // 1.5 2^23 + 128
+    int acc1[RPT];
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) {
+        const int p = rb + 16 * j;
+        const float xq = s_xqf[p], M = s_M[p];
+        const float2 xq2 = make_float2(xq, xq), M2 = make_float2(M, M);
+        const uint32_t hw[4] = {hw4[j].x, hw4[j].y, hw4[j].z, hw4[j].w};
+        uint32_t out[4];
+        int acc = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            acc = __dp4a((int)hw[q], cw[q], acc);                       // ChunkScan1 on the state before the token
+            // S8 = clamp(rint(float(xq bq) * M), +-127) for codes 4q .. 4q+3: xq bq is exact in fp32
+            uint32_t su[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float2 u = __fmul2_rn(__fmul2_rn(xq2, bqf[2 * q + e]), M2);
+                u.x = fminf(fmaxf(u.x, lim_lo.x), lim_hi.x);
+                u.y = fminf(fmaxf(u.y, lim_lo.y), lim_hi.y);
+                u = __fadd2_rn(u, rnd);                                  // bits 0x4B400000 + 128 + rint(u)
+                su[e] = __byte_perm(__float_as_uint(u.x), __float_as_uint(u.y), 0x5410);
+            }
+            if (packed) {
+                const uint32_t hu = hw[q] ^ 0x80808080u;
+                uint32_t v0 = __byte_perm(hu, 0, 0x4140) * (uint32_t)dq + k0x2 + (su[0] << k);
+                uint32_t v1 = __byte_perm(hu, 0, 0x4342) * (uint32_t)dq + k0x2 + (su[1] << k);
+                v0 = min_u16x2(max_u16x2(v0, lo), hi) >> k;
+                v1 = min_u16x2(max_u16x2(v1, lo), hi) >> k;
+                out[q] = __byte_perm(v0, v1, 0x6420);
+            } else {
+                out[q] = 0;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int hs = (int)(int8_t)(hw[q] >> (8 * v));
+                    const int s8 = (int)((su[v >> 1] >> (16 * (v & 1))) & 0xffffu) - 128;
+                    const int hn = sat127(s8 + ((dq * hs + (1 << (k - 1))) >> k));
+                    out[q] |= ((uint32_t)hn & 0xffu) << (8 * v);
+                }
+            }
+        }
+        acc1[j] = acc;
+        sp[p * (N / 16)] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) acc1[j] = row_sum<8>(acc1[j]);
+    if (sub == 0) {
+        const float m = bf16_bits_to_float(float_to_bf16_bits((float)cb * (sC * sB) * dtv));
+        const float ea = s_ea, Dh = __ldg(D + h);
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+            const int p = rb + 16 * j;
+            const float xv = s_xv[p];
+            const float y_o = (float)acc1[j] * s_ys[p] * ea;
+            y[bh * P + p] = float_to_bf16_bits(fmaf(Dh, xv, fmaf(m, xv, y_o)));
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_decode_bf16(const Dims& d, const uint16_t* x, const float* dt, const float* A, const uint16_t* B,
@@ -215,7 +355,13 @@ cudaError_t launch_decode_bf16(const Dims& d, const uint16_t* x, const float* dt
 cudaError_t launch_decode_i8(const Dims& d, const uint16_t* x, const float* dt, const float* A, const uint16_t* Bq,
                              const uint16_t* Cq, const float* D, const I8Scales& sc, int8_t* state, uint16_t* y,
                              cudaStream_t st) {
-    // N = 128 (P = 64): 2 rows per lane group, 8 rows of one head per warp (measured best of 1, 2, 4); N = 16: one row
+    const long long heads = (long long)d.B * d.H;
+    if (d.N == 128 && d.P == 64) {
+        if (heads == 0) return cudaSuccess;
+        decode_i8_head_kernel<<<(unsigned)heads, kHeadThreads, 0, st>>>(d, x, dt, A, Bq, Cq, D, sc, state, y);
+        return cudaGetLastError();
+    }
+    // other P with N = 128: 2 rows per lane group, 8 rows of one head per warp; N = 16: one row
     constexpr int kRpt128 = 2;
     if (d.N == 128 && d.P % (4 * kRpt128) != 0) return cudaErrorInvalidValue;
     const long long threads = (long long)d.B * d.H * d.P * (d.N / 16) / (d.N == 128 ? kRpt128 : 1);

@@ -187,16 +187,6 @@ __device__ __forceinline__ void red_release_add(int* p, int v) {
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -592,7 +582,7 @@ ssd_fused_i8_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             const int t = item_get(n);
             if (t < 0) break;
             const Item it = item_of(a, t);
-            const float sCB = __ldg(a.sc.s_C + it.g) * __ldg(a.sc.s_B + it.g);
+            const float sCB = __fmul_rn(__ldg(a.sc.s_C + it.g), __ldg(a.sc.s_B + it.g));
             bool ok = true;
             for (int hh = 0; hh < it.nh; ++hh, ++hk) {
                 const int h = it.h0 + hh, ss = hk % kNS, cs = hk % kNC;
@@ -643,7 +633,7 @@ ssd_fused_i8_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     for (int i = 0; i < m; ++i) dst[i] = acs[i];
                 }
                 // a2 at the end of the 32-element block of this lane's elements
-                const float ar = __shfl_sync(0xffffffffu, acs[m - 1] * kLog2e, lane | (32 / m - 1));
+                const float ar = __shfl_sync(0xffffffffu, __fmul_rn(acs[m - 1], kLog2e), lane | (32 / m - 1));
                 __syncwarp();
 #pragma unroll 1
                 for (int i = 0; i < m; i += 2) {
@@ -652,13 +642,15 @@ ssd_fused_i8_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     const float t0 = cvp[K::CV_DTW / 4 + j], t1 = cvp[K::CV_DTW / 4 + j + 1];
                     svp[K::SV_LUT / 4 + j] = __fmul_rn(t0, ssd_expf_call(__fsub_rn(last, c0v)));
                     svp[K::SV_LUT / 4 + j + 1] = __fmul_rn(t1, ssd_expf_call(__fsub_rn(last, c1v)));
-                    const float a0v = c0v * kLog2e, a1v = c1v * kLog2e;
-                    const float dw0 = t0 * sCB, dw1 = t1 * sCB;
+                    // explicitly rounded steps (no contraction), as in the five-launch ChunkScan
+                    const float a0v = __fmul_rn(c0v, kLog2e), a1v = __fmul_rn(c1v, kLog2e);
+                    const float dw0 = __fmul_rn(t0, sCB), dw1 = __fmul_rn(t1, sCB);
                     cvp[K::CV_A2 / 4 + j] = a0v;
                     cvp[K::CV_A2 / 4 + j + 1] = a1v;
-                    cvp[K::CV_DTW / 4 + j] = lg2(dw0) - a0v;
-                    cvp[K::CV_DTW / 4 + j + 1] = lg2(dw1) - a1v;
-                    const float v0 = ex2(fminf(ar - a0v, 0.f)) * dw0, v1 = ex2(fminf(ar - a1v, 0.f)) * dw1;
+                    cvp[K::CV_DTW / 4 + j] = __fsub_rn(lg2(dw0), a0v);
+                    cvp[K::CV_DTW / 4 + j + 1] = __fsub_rn(lg2(dw1), a1v);
+                    const float v0 = __fmul_rn(ex2(fminf(__fsub_rn(ar, a0v), 0.f)), dw0);
+                    const float v1 = __fmul_rn(ex2(fminf(__fsub_rn(ar, a1v), 0.f)), dw1);
                     reinterpret_cast<uint32_t*>(cvp + K::CV_VB / 4)[j / 2] = pack_bf16(v0, v1);
                 }
                 if (lane == 31) {

@@ -12,6 +12,16 @@ TOL_BF16 = 5e-3        # relative L2 of y and the final state against fp64
 TOL_I8_Y = 5e-2        # relative L2 of the dequantised W8A8 y against fp64
 
 
+def poison(torch, pb) -> None:
+    """Fill an SsdProblem's outputs with values no kernel produces: NaN bit patterns in y and
+    the fp32 state, code -128 in the INT8 state."""
+    pb.y.view(torch.int16).fill_(-1)
+    if getattr(pb, "final32", None) is not None:
+        pb.final32.fill_(float("nan"))
+    if getattr(pb, "final8", None) is not None:
+        pb.final8.fill_(-128)
+
+
 def bf16_to_np(t) -> np.ndarray:
     """float64 values of a bf16 torch tensor."""
     import torch

@@ -83,8 +83,10 @@ def test_bf16_decode_continues_a_scan(torch_cuda):
     assert rel_l2(host(dec.state).astype(np.float64), ef) <= TOL_BF16
 
 
-@pytest.mark.parametrize("name", list(CASES))
-def test_i8_decode_steps_bit_exact(torch_cuda, name):
+@pytest.mark.parametrize("name,shift", [("2.7b-shape", 7), ("2.7b-shape", 5), ("2.7b-shape", 9), ("small", 7)])
+def test_i8_decode_steps_bit_exact(torch_cuda, name, shift):
+    """Shifts 5 and 7 take the (P, N) = (64, 128) kernel's two-codes-per-word carry, 9 its
+    code-at-a-time one; the (16, 16) shape runs the row kernel."""
     torch = torch_cuda
     from int8_quant_b200.runner import Decoder, to_device
     w = CASES[name]
@@ -93,7 +95,7 @@ def test_i8_decode_steps_bit_exact(torch_cuda, name):
     sc = oracle_scales(inp, w.chunk, w.calib_prefix)
     scd = {k: torch.from_numpy(np.asarray(v, F32)).cuda() for k, v in sc.items() if k.startswith("s_")}
     st8 = np.random.default_rng(4).integers(-90, 91, (w.batch, w.nheads, w.headdim, w.dstate)).astype(np.int8)
-    dec = Decoder(torch.from_numpy(st8.copy()).cuda(), dev["A"], dev["D"], "w8a8", scd)
+    dec = Decoder(torch.from_numpy(st8.copy()).cuda(), dev["A"], dev["D"], "w8a8", scd, shift=shift)
     x, Bv, Cv = as_float(inp["x"]).astype(F32), as_float(inp["B"]).astype(F32), as_float(inp["C"]).astype(F32)
     Bq, Cq = W.quantize_inputs(Bv, Cv, sc["s_B"], sc["s_C"])
     ref = st8
@@ -102,10 +104,12 @@ def test_i8_decode_steps_bit_exact(torch_cuda, name):
         y = bf16_to_np(dec.step(tk["x"], tk["dt"], tk["B"], tk["C"]).clone())
         torch.cuda.synchronize()
         r = W.decode_step_i8(x[:, t], inp["dt"][:, t], inp["A"], Bq[:, t], Cq[:, t], inp["D"], sc["s_B"], sc["s_C"],
-                             sc["s_x"], sc["s_s"], ref)
+                             sc["s_x"], sc["s_s"], ref, k=shift)
         np.testing.assert_array_equal(host(dec.state), r["state8"])
         assert rel_l2(y, r["y"]) <= 1e-2, (t, rel_l2(y, r["y"]))
         ref = r["state8"]
+    if shift != 7:                                  # coarser or finer decay codes: the integers decide
+        return
     H, P = w.nheads, w.headdim
     ss = np.asarray(sc["s_s"], np.float64).reshape(H, P)[None, :, :, None]
     ey, _ = F.ssd_sequential(as_float(inp["x"])[:, :8], inp["dt"][:, :8], inp["A"], as_float(inp["B"])[:, :8],

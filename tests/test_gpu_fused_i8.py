@@ -19,7 +19,7 @@ from harness import Workload, WORKLOADS, make_inputs, as_float
 from oracle import ssd_w8a8 as W
 from oracle.ssd_fp64 import rel_l2
 from tests.gpu_common import (TOL_I8_Y, bf16_to_np, host, oracle_fp64, oracle_i8, oracle_scales, chain_oracle,
-                              chain_oracle_i8, full_size_scales)
+                              chain_oracle_i8, full_size_scales, poison)
 
 pytestmark = pytest.mark.gpu
 
@@ -29,6 +29,7 @@ CASES = {
     "ragged-q64": Workload("ragged-q64", 2, 333, 4, 64, 128, 4, 64, seed=2),
     "L1": Workload("L1", 2, 1, 4, 64, 128, 1, 256, seed=4),
     "ragged-heads": Workload("ragged-heads", 1, 512, 20, 64, 128, 1, 256, seed=6),
+    "g1-ragged": Workload("g1-ragged", 2, 1000, 6, 64, 128, 1, 256, seed=7, head_scale=True, outliers=True),
 }
 F32 = np.float32
 
@@ -44,9 +45,12 @@ def fused(monkeypatch):
 
 
 def _problem(w, inp=None):
+    import torch
     from int8_quant_b200.runner import SsdProblem, to_device
     inp = make_inputs(w) if inp is None else inp
-    return inp, SsdProblem(to_device(inp), w.chunk, with_bf16=False)
+    pb = SsdProblem(to_device(inp), w.chunk, with_bf16=False)
+    poison(torch, pb)
+    return inp, pb
 
 
 def _check_against_oracle(torch, w, shift=7):
@@ -85,24 +89,27 @@ def test_fused_other_decay_shifts(fused, shift):
     _check_against_oracle(fused, CASES["ragged-q256"], shift)
 
 
-@pytest.mark.parametrize("name", ["ragged-q256", "ragged-q64", "ragged-heads"])
+@pytest.mark.parametrize("name", ["ragged-q256", "ragged-q64", "ragged-heads", "g1-ragged"])
 def test_fused_equals_staged(fused, name, monkeypatch):
-    """Same y and final state, bit for bit, as the five-launch path."""
+    """Same y and final state, bit for bit, as the five-launch path; every output written
+    (y starts as NaN bit patterns, the state as an out-of-range code, before each run)."""
     torch = fused
     w = CASES[name]
     inp, pb = _problem(w)
     sc = oracle_scales(inp, w.chunk, w.calib_prefix)
     pb.set_scales(sc["s_B"], sc["s_C"], sc["s_x"], sc["s_s"], 7)
-    pb.run_i8()
-    torch.cuda.synchronize()
-    y_f, fin_f = pb.y.clone(), pb.final8.clone()
-    monkeypatch.setenv("SSD_I8_FUSED", "0")
-    pb.y.zero_()
-    pb.final8.zero_()
-    pb.run_i8()
-    torch.cuda.synchronize()
-    assert torch.equal(fin_f, pb.final8)
-    assert torch.equal(y_f.view(torch.int16), pb.y.view(torch.int16))
+    out = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("SSD_I8_FUSED", flag)
+        pb.y.view(torch.int16).fill_(-1)
+        pb.final8.fill_(-128)
+        pb.run_i8()
+        torch.cuda.synchronize()
+        out.append((pb.y.view(torch.int16).clone(), pb.final8.clone()))
+    for y, fin in out:
+        assert not bool((y == -1).any()) and not bool((fin == -128).any())
+    assert torch.equal(out[0][1], out[1][1])
+    assert torch.equal(out[0][0], out[1][0]), int((out[0][0] != out[1][0]).sum())
 
 
 def test_fused_production_equals_debug(fused):

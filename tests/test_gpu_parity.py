@@ -10,7 +10,7 @@ import pytest
 
 from harness import Workload, WORKLOADS, make_inputs
 from oracle.ssd_fp64 import rel_l2
-from tests.gpu_common import (TOL_BF16, TOL_I8_Y, bf16_to_np, host, oracle_fp64, oracle_i8, oracle_scales)
+from tests.gpu_common import (TOL_BF16, TOL_I8_Y, bf16_to_np, host, oracle_fp64, oracle_i8, oracle_scales, poison)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,9 +37,13 @@ def torch_cuda():
 
 
 def _problem(torch_cuda, w):
+    """Inputs and device buffers; the outputs start as NaN bit patterns (y, fp32 state) and
+    code -128 (INT8 state), so that an element the kernels never write fails the checks."""
     from int8_quant_b200.runner import SsdProblem, to_device
     inp = make_inputs(w)
-    return inp, SsdProblem(to_device(inp), w.chunk)
+    pb = SsdProblem(to_device(inp), w.chunk)
+    poison(torch_cuda, pb)
+    return inp, pb
 
 
 @pytest.mark.parametrize("name", list(CASES))
