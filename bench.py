@@ -145,17 +145,19 @@ def measured_bf16_tflops() -> float:
 # capture, keyed by kernel name, with the sha1 of the kernel source it was taken on.
 # A kernel whose source changed since reports null.
 NCU_TRAFFIC = {
-    # batch-2 capture scaled x4 to the batch-8 launch (traffic grows with the batch)
-    ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.510976e6 + 131.441664e6),
-                                            "src_sha1": "d4289772c1f95756fab8af3deacde1b311a52d75"},
-    ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (270.597632e6 + 133.411328e6),
-                                            "src_sha1": "d4289772c1f95756fab8af3deacde1b311a52d75"},
+    # batch-2 captures scaled x4 to the batch-8 launch (traffic grows with the batch)
+    ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.53e6 + 124.93e6),
+                                            "src_sha1": "6936eeb314b08b35b182d306bf9dc82023da0330"},
+    ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (270.60e6 + 128.12e6),
+                                            "src_sha1": "6936eeb314b08b35b182d306bf9dc82023da0330"},
+    ("ssd_fused_i8", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (178.17e6 + 176.30e6),
+                                              "src_sha1": "3a08a823dcfb46ab30d6bebff0bd7ab1e004d1e8"},
 }
 
 
 def _src_hash(kernel: str):
     f = {"chunk_scan": "chunk_scan_tc.cu", "chunk_state": "chunk_state_tc.cu", "state_passing": "state_passing.cu",
-         "chunk_cumsum": "cumsum.cu", "quantize_inputs": "quantize.cu"}.get(kernel)
+         "chunk_cumsum": "cumsum.cu", "quantize_inputs": "quantize.cu", "ssd_fused_i8": "fused_i8.cu"}.get(kernel)
     if not f:
         return None
     with open(os.path.join(ROOT, "int8_quant_b200", "csrc", f), "rb") as fh:
@@ -348,6 +350,16 @@ def replica_throughput(tokens_per_rank: int, ms_per_step: float, world: int) -> 
     return world * tokens_per_rank / (ms_per_step / 1e3)
 
 
+# kernels each profiled stage launches (the single-launch scan's stage also runs the
+# small kernel that forms its per-(h,p) factors)
+KERNELS_PER_STAGE = {"ssd_fused_i8": 2}
+
+
+def kernel_launches(kern) -> int:
+    """This library's kernel launches behind the per-stage counts of ssd_profile_read."""
+    return sum(c * KERNELS_PER_STAGE.get(k, 1) for k, (_, c) in kern.items())
+
+
 def tc_shape(w) -> bool:
     """(P, N) = (64, 128): the shape the tensor-core kernels (and the single-launch scan) take."""
     return (w.headdim, w.dstate) == (64, 128)
@@ -436,42 +448,68 @@ def run_ours(args, rank, world, dist):
                 "frac_of_measured_hbm": round(alg / t / 1e9 / peak, 4),
                 "frac_of_8TBs": round(alg / t / 1e9 / DATASHEET_HBM_GBS, 4)}
 
-    def decode(path, steps=50, warm=5):
-        """One-token steps continuing the scan's final state (ssd_decode_step_*, one launch
-        per token; W8A8 quantises the token's B and C inside).  L2 is refilled with other
-        data before every step (a read of 256 MB, which leaves no dirty lines to write
-        back), so each step reads and writes the whole state from HBM, as it would between
-        the other layers of a model; the time is the decode kernel's own (CUDA events
-        around each launch), not the refill."""
+    def decode_time(path, state, toks, steps, warm):
+        """Average decode-kernel time (µs) over `steps` one-token steps, L2 refilled before each."""
         from int8_quant_b200.runner import Decoder
-        state = (pb.final8 if path == "w8a8" else pb.final32).clone()
         dec = Decoder(state, dinp["A"], dinp["D"], path, pb.scales if path == "w8a8" else None)
-        toks = [{k: dinp[k][:, t].contiguous() for k in ("x", "dt", "B", "C")} for t in range(8)]
         flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
         for i in range(warm):
-            dec.step(**toks[i % 8], stream=stream)
+            dec.step(**toks[i % len(toks)], stream=stream)
         torch.cuda.synchronize()
         iq.ssd_profile_reset()
         for i in range(steps):
             with torch.cuda.stream(stream):
                 flush.amax()
             iq.ssd_profile_enable(True)
-            dec.step(**toks[i % 8], stream=stream)
+            dec.step(**toks[i % len(toks)], stream=stream)
             iq.ssd_profile_enable(False)
         torch.cuda.synchronize()
         kern = iq.ssd_profile_read()
-        us = {k: v[0] / max(v[1], 1) * 1e3 for k, v in kern.items()}
-        step_us = sum(us.values())
-        b, H, P, N, G = w.batch, w.nheads, w.headdim, w.dstate, w.ngroups
+        return {k: v[0] / max(v[1], 1) * 1e3 for k, v in kern.items()}
+
+    def decode_bytes(path, b):
+        H, P, N, G = w.nheads, w.headdim, w.dstate, w.ngroups
         eb = 1 if path == "w8a8" else 4
-        alg = b * H * P * N * eb * 2 + b * H * P * 4 + b * H * 4 + b * G * N * 4
+        return b * H * P * N * eb * 2 + b * H * P * 4 + b * H * 4 + b * G * N * 4
+
+    def decode(path, steps=50, warm=5):
+        """One-token steps continuing the scan's final state (ssd_decode_step_*, one launch
+        per token; W8A8 quantises the token's B and C inside).  L2 is refilled with other
+        data before every step (a read of 256 MB, which leaves no dirty lines to write
+        back), so each step reads and writes the whole state from HBM, as it would between
+        the other layers of a model; the time is the decode kernel's own (CUDA events
+        around each launch), not the refill.  `batch_sweep` repeats the step at larger
+        batches (synthetic tokens of the same recipe, a random state) to separate the
+        per-launch floor from the per-byte cost."""
+        state = (pb.final8 if path == "w8a8" else pb.final32).clone()
+        toks = [{k: dinp[k][:, t].contiguous() for k in ("x", "dt", "B", "C")} for t in range(8)]
+        us = decode_time(path, state, toks, steps, warm)
+        step_us = sum(us.values())
+        b = w.batch
+        alg = decode_bytes(path, b)
         k_us = us.get("decode_step", 0.0)
+        sweep = {}
+        g = torch.Generator(device=dev).manual_seed(11)
+        for bb in (32, 128):
+            ti = to_device(make_inputs(w.with_(batch=bb, seqlen=8)), dev)
+            tk = [{k: ti[k][:, t].contiguous() for k in ("x", "dt", "B", "C")} for t in range(8)]
+            shp = (bb, w.nheads, w.headdim, w.dstate)
+            st = (torch.randint(-90, 91, shp, generator=g, device=dev, dtype=torch.int8) if path == "w8a8"
+                  else torch.randn(shp, generator=g, device=dev))
+            t_us = decode_time(path, st, tk, 20, 3).get("decode_step", 0.0)
+            ab = decode_bytes(path, bb)
+            sweep[str(bb)] = {"us": round(t_us, 3), "alg_bytes": ab,
+                              "achieved": round(ab / (t_us * 1e-6) / 1e9, 1) if t_us else None,
+                              "frac": round(ab / (t_us * 1e-6) / 1e9 / peak, 4) if t_us else None}
+            del ti, tk, st
         return {"tokens_per_s": round(b / (step_us * 1e-6), 1), "us_per_step": round(step_us, 3),
-                "kernels_us": {k: round(v, 3) for k, v in us.items()},
+                "kernels_us": {k: round(v, 3) for k, v in us.items() if v},
                 "roofline": {"kernel": "decode_step", "bound": "hbm", "alg_bytes": alg,
                              "achieved": round(alg / (k_us * 1e-6) / 1e9, 1) if k_us else None, "peak": peak,
                              "unit": "GB/s", "frac": round(alg / (k_us * 1e-6) / 1e9 / peak, 4) if k_us else None},
-                "state": f"{'int8' if path == 'w8a8' else 'fp32'} [{b},{H},{P},{N}], continuing the scan's final state",
+                "batch_sweep": sweep,
+                "state": f"{'int8' if path == 'w8a8' else 'fp32'} [{b},{w.nheads},{w.headdim},{w.dstate}], "
+                         "continuing the scan's final state",
                 "l2": "refilled with 256 MB of other reads before every step"}
 
     def out_proj(steps=10, warm=3):
@@ -558,7 +596,7 @@ def run_ours(args, rank, world, dist):
                 os.environ["SSD_I8_FUSED"] = old
         return {"value": replica_throughput(w.tokens, ms, world), "ms_per_step": round(ms, 5),
                 "roofline": roofline("w8a8", kern, w), "path_roofline": path_roofline("w8a8", ms, w),
-                "gpu_launches": sum(c for _, c in kern.values()), "clocks": clocks,
+                "gpu_launches": kernel_launches(kern), "clocks": clocks,
                 "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in kern.items()}}
 
     def other_config(name):
@@ -580,7 +618,7 @@ def run_ours(args, rank, world, dist):
             out[path] = {"value": replica_throughput(wo.tokens, ms, world), "ms_per_step": round(ms, 5),
                          "path_roofline": path_roofline(path, ms, wo),
                          "roofline": {k: rf[k] for k in ("kernel", "achieved", "frac", "frac_of_8TBs", "launch_ms")},
-                         "gpu_launches": sum(c for _, c in kern.values()), "clocks": clocks,
+                         "gpu_launches": kernel_launches(kern), "clocks": clocks,
                          "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in kern.items()}}
         if tc_shape(wo):
             out["w8a8_fused"] = {k: v for k, v in fused_i8(wo, po).items() if k != "kernels_ms_per_step"}
@@ -592,7 +630,7 @@ def run_ours(args, rank, world, dist):
     paths = (args.path,) if args.only_path else (args.path, "bf16" if args.path == "w8a8" else "w8a8")
     for path in paths:
         ms, kern, clocks = timed(path)
-        launches = sum(c for _, c in kern.values())
+        launches = kernel_launches(kern)
         results[path] = {
             "ms_per_step": ms, "value": replica_throughput(w.tokens, ms, world), "kern": kern, "clocks": clocks,
             "roofline": roofline(path, kern), "gpu_launches": launches,
