@@ -71,17 +71,21 @@ struct Cfg {
     static constexpr int H_BYTES = kP * kN * EB;
     static constexpr int NHB = kI8 ? 2 : 1;                      // state tile buffers
     static constexpr int X_BYTES = Q * 128;
+    // x stages (each also holds its head's y until the store has read it): three when
+    // shared memory allows, so that two heads' loads can be in flight ahead of the MMAs
+    static constexpr int NXS = kI8 ? 3 : 2;
     static constexpr int OFF_C = 0;
     static constexpr int OFF_B = C_BYTES;
     static constexpr int OFF_X = (OFF_B + B_BYTES + 1023) & ~1023;
-    static constexpr int OFF_H = OFF_X + 2 * X_BYTES;
+    static constexpr int OFF_H = OFF_X + NXS * X_BYTES;
     static constexpr int OFF_VEC = OFF_H + NHB * H_BYTES;        // 2 slots x {acs, dtc, a2, vB, dtw}[Q]
     static constexpr int VEC_SLOT = (kI8 ? 6 : 5) * Q * 4;
     static constexpr int OFF_BAR = OFF_VEC + 2 * VEC_SLOT;
     // barriers
-    static constexpr int B_LOAD = 0, B_CB = 1, B_PACKED = 2, B_XFULL = 3, B_XEMPTY = 5, B_HFULL = 7,
-                         B_HEMPTY = 9, B_VFULL = 11, B_VEMPTY = 13, B_RFULL = 15, B_REMPTY = 15 + kRing,
-                         B_YOFULL = 15 + 2 * kRing, B_YSCALED = B_YOFULL + 2, B_YFULL = B_YOFULL + 4,
+    static constexpr int B_LOAD = 0, B_CB = 1, B_PACKED = 2, B_XFULL = 3, B_XEMPTY = 3 + NXS,
+                         B_HFULL = 3 + 2 * NXS, B_HEMPTY = B_HFULL + 2, B_VFULL = B_HEMPTY + 2,
+                         B_VEMPTY = B_VFULL + 2, B_RFULL = B_VEMPTY + 2, B_REMPTY = B_RFULL + kRing,
+                         B_YOFULL = B_RFULL + 2 * kRing, B_YSCALED = B_YOFULL + 2, B_YFULL = B_YOFULL + 4,
                          B_YEMPTY = B_YOFULL + 6, B_VPREP = B_YOFULL + 8, NBAR = B_YOFULL + 10;
     static constexpr int OFF_FLAG = OFF_BAR + NBAR * 8;
     static constexpr int OFF_TMEM = OFF_FLAG + 8;
@@ -257,9 +261,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 uint8_t* hdst = sm + K::OFF_H + hb * K::H_BYTES;
                 tc::tma_load_2d(hdst, &tm_h, bar + K::B_HFULL + hb, 0, hrow);
                 if (!kI8) tc::tma_load_2d(hdst + kP * 128, &tm_h, bar + K::B_HFULL + hb, 64, hrow);
-                if (!wait_bar<kI8>(bar + K::B_XEMPTY + s, (u & 1) ^ 1, abort_flag, status)) break;
-                tc::mbar_arrive_expect_tx(bar + K::B_XFULL + s, K::X_BYTES);
-                tc::tma_load_3d(sm + K::OFF_X + s * K::X_BYTES, &tm_x, bar + K::B_XFULL + s, h * kP, c * Q, b);
+                const int xst = it % K::NXS;
+                const uint32_t xu = (uint32_t)(it / K::NXS);
+                if (!wait_bar<kI8>(bar + K::B_XEMPTY + xst, (xu & 1) ^ 1, abort_flag, status)) break;
+                tc::mbar_arrive_expect_tx(bar + K::B_XFULL + xst, K::X_BYTES);
+                tc::tma_load_3d(sm + K::OFF_X + xst * K::X_BYTES, &tm_x, bar + K::B_XFULL + xst, h * kP, c * Q, b);
             }
         }
     } else if (warp == 1) {
@@ -358,8 +364,9 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             // the builders share this warp's scheduler)
             if (yo == it + 1 && yo < nh && !(ok = issue_yo(false))) break;
             if (!(ok = wait_all(K::B_YSCALED + s, u & 1))) break;
-            if (!(ok = wait_all(K::B_XFULL + s, u & 1))) break;
-            const uint64_t dX = dX0 + (uint64_t)((s * K::X_BYTES) >> 4);
+            const int xst = it % K::NXS;
+            if (!(ok = wait_all(K::B_XFULL + xst, (uint32_t)(it / K::NXS) & 1))) break;
+            const uint64_t dX = dX0 + (uint64_t)((xst * K::X_BYTES) >> 4);
             const uint32_t ycol = tmem + K::YCOL + 128 * s;
             for (int k = 0; k < K::NPIECE; ++k, ++p) {
                 int J, ib;
@@ -641,11 +648,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         for (int it = 0; ok && it < nh; ++it) {
             const int h = h0 + it, s = it & 1;
             const uint32_t u = (uint32_t)(it >> 1);
+            const int xst = it % K::NXS;
             bool w = wait_bar<kI8>(bar + K::B_YFULL + s, u & 1, abort_flag, status);
-            w = w && wait_bar<kI8>(bar + K::B_XFULL + s, u & 1, abort_flag, status);
+            w = w && wait_bar<kI8>(bar + K::B_XFULL + xst, (uint32_t)(it / K::NXS) & 1, abort_flag, status);
             if (!(ok = tc::named_and(kIdStore, kEpiThreads, w))) break;
             tc::tc_fence_after();
-            uint8_t* xs = sm + K::OFF_X + s * K::X_BYTES;
+            uint8_t* xs = sm + K::OFF_X + xst * K::X_BYTES;
             const uint32_t ybase = trow + K::YCOL + 128 * s;
             const float Dh = __ldg(Dv + h);
             for (int J = 0; J < K::JT; ++J) {
@@ -684,7 +692,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 tc::tma_store_3d(&tm_y, xs, h * kP, c * Q, b);
                 tc::tma_store_commit();
                 tc::tma_store_wait_read0();
-                tc::mbar_arrive(bar + K::B_XEMPTY + s);
+                tc::mbar_arrive(bar + K::B_XEMPTY + xst);
             }
         }
         if (warp == kStoreWarp0 && lane == 0) tc::tma_store_wait0();
