@@ -393,24 +393,31 @@ def run_ours(args, rank, world, dist):
             dist.barrier()
 
     def timed(path, pb=pb):
+        """Step time over the timed loop (CUDA events around all steps, no per-kernel events,
+        so consecutive launches may overlap as they do in use), then the per-kernel split
+        from a second, profiled pass of the same number of steps (an event pair around every
+        kernel)."""
         step = step_fn(path, pb)
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize()
-        iq.ssd_profile_reset()
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with ClockSampler(dev) as clk:
             barrier()
             torch.cuda.synchronize()
-            iq.ssd_profile_enable(True)
             ev0.record(stream)
             for _ in range(args.steps):
                 step()
             ev1.record(stream)
             torch.cuda.synchronize()
-            iq.ssd_profile_enable(False)
             barrier()
         ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev) / args.steps
+        iq.ssd_profile_reset()
+        iq.ssd_profile_enable(True)
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize()
+        iq.ssd_profile_enable(False)
         kern = iq.ssd_profile_read()
         return ms, kern, clk.summary()
 
