@@ -606,6 +606,21 @@ def run_ours(args, rank, world, dist):
                 "gpu_launches": kernel_launches(kern), "clocks": clocks,
                 "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in kern.items()}}
 
+    def storage_variant(w=w, pb=pb):
+        """The W8A8 step with the notes' storage variant (Acs as FP16, CB requantised to INT8
+        tiles in HBM by a ChunkBMM kernel and read back by ChunkScan2), timed the same way;
+        its DRAM traffic is measured with ncu (the bytes it adds are intermediates, so the
+        path roofline's compulsory bytes are the same)."""
+        pb.set_storage(iq.SSD_STORAGE_ACS_FP16 | iq.SSD_STORAGE_CB_INT8)
+        try:
+            ms, kern, clocks = timed("w8a8", pb)
+        finally:
+            pb.set_storage(0)
+        return {"value": replica_throughput(w.tokens, ms, world), "ms_per_step": round(ms, 5),
+                "path_roofline": path_roofline("w8a8", ms, w), "gpu_launches": kernel_launches(kern),
+                "clocks": clocks, "kernels_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in kern.items()},
+                "storage": "Acs FP16 + CB INT8 in HBM (SSD_STORAGE_ACS_FP16 | SSD_STORAGE_CB_INT8)"}
+
     def other_config(name):
         """Device-timed step of another workload on both paths (its own inputs, calibrated the
         same way); no e2e, decode or epilogue."""
@@ -647,6 +662,8 @@ def run_ours(args, rank, world, dist):
             results[path]["e2e"] = e2e(path)
     if "w8a8" in paths and tc_shape(w) and not args.no_fused:
         results["w8a8_fused"] = fused_i8()
+    if "w8a8" in paths and tc_shape(w) and w.chunk == 256 and not args.no_storage_variant:
+        results["w8a8_notes_storage"] = storage_variant()
     if not args.no_decode:
         results["decode"] = {p: decode(p) for p in paths}
     if not args.no_out_proj:
@@ -671,6 +688,8 @@ def main():
     ap.add_argument("--seqlen", type=int, default=None, help="override the workload's length (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fused", action="store_true", help="skip the single-launch W8A8 scan measurement")
+    ap.add_argument("--no-storage-variant", action="store_true",
+                    help="skip the W8A8 step with the notes' storage variant (FP16 Acs, INT8 CB in HBM)")
     ap.add_argument("--all-configs", action="store_true",
                     help="also time every other workload on both paths (device time only; adds minutes)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -758,6 +777,8 @@ def main():
     }
     if "w8a8_fused" in res:
         line["w8a8_fused"] = res["w8a8_fused"]
+    if "w8a8_notes_storage" in res:
+        line["w8a8_notes_storage"] = res["w8a8_notes_storage"]
     if "configs" in res:
         line["configs"] = res["configs"]
     if "decode" in res:

@@ -85,7 +85,20 @@ typedef struct {
     const float* s_x;      /* [H*P], scale of X_scaled = LUT_state ⊙ x */
     const float* s_s;      /* [H*P], scale of the INT8 state */
     int decay_shift;       /* k of eq. 6 (S = 2^k); 1..14, the notes use 7 */
+    int storage;           /* 0: the library's layout (Acs fp32, CB kept on chip as INT32);
+                            * otherwise flags of the notes' storage variant (overall
+                            * framework; key design 2), for measurement and study:
+                            * SSD_STORAGE_ACS_FP16 keeps Acs as IEEE half (every use reads
+                            * the half value), SSD_STORAGE_CB_INT8 requantises each (b, c, g)
+                            * CB tile to INT8 with one step amax|CB| / 127 (fp64; amax 0
+                            * gives 1) and writes the codes to the workspace, from which
+                            * ChunkScan2 reads them.  Flags need (P, N) = (64, 128) and
+                            * chunk 256 (else SSD_ERR_UNSUPPORTED) and run the five-launch
+                            * pipeline.  Zero-initialise the struct for the default. */
 } ssd_i8_params;
+
+#define SSD_STORAGE_ACS_FP16 1
+#define SSD_STORAGE_CB_INT8 2
 
 /* Human-readable name of a status code (static string). */
 const char* ssd_status_string(ssd_status s);
@@ -188,8 +201,11 @@ ssd_status ssd_scan_fwd_i8(const ssd_shape* shape, const uint16_t* x, const floa
  *   acc_state int32 [B, nc, H, P, N]  ChunkState accumulator Q(X_scaled)^T Q(B)
  *   S8        int8  [B, nc, H, P, N]  requantised chunk states
  *   H8        int8  [B, nc, H, P, N]  INT8 state entering each chunk
- *   cb        int32 [B, nc, G, Q, Q]  ChunkBMM accumulator Cq Bq^T (entries with i <= j)
- *   acc_scan1 int32 [B, Lp, H, P]     ChunkScan1 accumulator Cq H8^T */
+ *   cb        int32 [B, nc, G, Q, Q]  ChunkBMM accumulator Cq Bq^T (entries with i <= j;
+ *                                     every entry with SSD_STORAGE_CB_INT8)
+ *   acc_scan1 int32 [B, Lp, H, P]     ChunkScan1 accumulator Cq H8^T
+ *   cb8       int8  [B, nc, G, Q, Q]  SSD_STORAGE_CB_INT8 only: the CB codes
+ *   s_cb      fp64  [B, nc, G]        SSD_STORAGE_CB_INT8 only: their steps */
 typedef struct {
     float* Acs;
     int32_t* dq;
@@ -199,6 +215,8 @@ typedef struct {
     int8_t* H8;
     int32_t* cb;
     int32_t* acc_scan1;
+    int8_t* cb8;
+    double* s_cb;
 } ssd_i8_debug;
 
 /* ssd_scan_fwd_i8 continuing from a given INT8 state: initial_state is device int8

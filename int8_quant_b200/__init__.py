@@ -4,6 +4,7 @@ The compute lives in libssd.so (hand-written CUDA); `ssd` is its ctypes binding 
 `runner` allocates device buffers with torch and sequences the calls.
 """
 from .ssd import (SsdShape, SsdI8Params, SsdError, library, shape_of, i8_params,  # noqa: F401
+                  SSD_STORAGE_ACS_FP16, SSD_STORAGE_CB_INT8,
                   ssd_workspace_bytes, ssd_calibrate_workspace_bytes, ssd_quantize_inputs,
                   ssd_scan_fwd_bf16, ssd_scan_fwd_bf16_static, ssd_static_scratch_status, ssd_scan_fwd_i8, ssd_scan_fwd_i8_debug, ssd_calibrate_i8,
                   ssd_workspace_status, ssd_profile_enable, ssd_profile_read, ssd_profile_reset,

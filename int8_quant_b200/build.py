@@ -10,7 +10,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libssd.so")
 SOURCES = ["api.cu", "quantize.cu", "cumsum.cu", "chunk_state.cu", "state_passing.cu", "chunk_scan.cu",
            "noalloc.cu", "tmap.cu", "chunk_state_tc.cu", "chunk_scan_tc.cu", "selftest.cu",
-           "decode.cu", "out_proj.cu", "fused_i8.cu"]
+           "decode.cu", "out_proj.cu", "fused_i8.cu", "chunk_bmm.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared"]
 

@@ -128,6 +128,8 @@ WsLayout ws_layout(const Dims& d, bool i8, bool fp32_states) {
     w.states = off;  off += align256(states * s_elem);
     w.passed = off;  off += align256(states * (i8 ? 1 : sizeof(uint16_t)));
     w.scales = off;  off += align256(i8 ? (size_t)2 * d.H * d.P * sizeof(float) : 0);   // 1/s_x, s_x s_B / s_s
+    // the storage variant's CB codes and steps (W8A8, tensor-core shape, chunk 256)
+    w.cb8 = off;     off += (i8 && tensor_core_shape(d) && d.Q == 256) ? align256(chunk_bmm_i8_bytes(d)) : 0;
     w.total = off;
     return w;
 }
@@ -320,6 +322,10 @@ static ssd_status scan_i8(const ssd_shape* shape, const uint16_t* x, const float
     if (st != SSD_OK) return st;
     if (!params || !params->s_B || !params->s_C || !params->s_x || !params->s_s) return SSD_ERR_INVALID_ARG;
     if (params->decay_shift < 1 || params->decay_shift > 14) return SSD_ERR_INVALID_ARG;
+    const int storage = params->storage;
+    if (storage & ~(SSD_STORAGE_ACS_FP16 | SSD_STORAGE_CB_INT8)) return SSD_ERR_INVALID_ARG;
+    if (storage && (!tensor_core_shape(d) || d.Q != 256)) return SSD_ERR_UNSUPPORTED;
+    const bool acs_half = (storage & SSD_STORAGE_ACS_FP16) != 0, cb_int8 = (storage & SSD_STORAGE_CB_INT8) != 0;
     if (d.B == 0) return SSD_OK;
     st = check_common(d, x, dt, A, Bq, Cq, D, y, final_state, workspace, workspace_bytes, true);
     if (st != SSD_OK) return st;
@@ -334,8 +340,10 @@ static ssd_status scan_i8(const ssd_shape* shape, const uint16_t* x, const float
     }
     I8Scales sc{params->s_B, params->s_C, params->s_x, params->s_s, params->decay_shift};
     I8Debug dd{};
-    if (dbg) dd = I8Debug{dbg->Acs, dbg->dq, dbg->Xq, dbg->acc_state, dbg->S8, dbg->H8, dbg->cb, dbg->acc_scan1};
-    if (i8_fused(d)) {
+    if (dbg)
+        dd = I8Debug{dbg->Acs, dbg->dq, dbg->Xq, dbg->acc_state, dbg->S8, dbg->H8, dbg->cb, dbg->acc_scan1,
+                     dbg->cb8, dbg->s_cb};
+    if (i8_fused(d) && !storage) {
         SSD_STAGE("ssd_fused_i8", launch_fused_i8(d, x, dt, A, Bq, Cq, D, sc, initial_state, y, final_state, workspace,
                                                   dbg ? &dd : nullptr, stream));
         return SSD_OK;
@@ -349,22 +357,29 @@ static ssd_status scan_i8(const ssd_shape* shape, const uint16_t* x, const float
     int* status = at<int>(workspace, w.status);
     float* inv_sx = at<float>(workspace, w.scales);
     float* mq = inv_sx + d.H * d.P;
-    SSD_STAGE("chunk_cumsum", launch_cumsum(d, dt, A, Acs, nullptr, dq, sc.shift, status, lut, dtc, stream, &sc, inv_sx, mq));
+    SSD_STAGE("chunk_cumsum", launch_cumsum(d, dt, A, Acs, nullptr, dq, sc.shift, status, lut, dtc, stream, &sc, inv_sx, mq,
+                                            acs_half));
     if (tensor_core_shape(d))
         SSD_STAGE("chunk_state", launch_chunk_state_tc(d, true, x, Bq, lut, inv_sx, mq, nullptr, S8, dbg ? &dd : nullptr,
                                                        status, stream));
     else
         SSD_STAGE("chunk_state", launch_chunk_state_i8(d, x, dt, Acs, Bq, sc, S8, dbg ? &dd : nullptr, stream));
     SSD_STAGE("state_passing", launch_state_passing_i8(d, S8, dq, sc.shift, initial_state, H8, final_state, stream));
+    int8_t* cb8 = at<int8_t>(workspace, w.cb8);
+    float* s_cb = at<float>(workspace, w.cb8 + (size_t)d.B * d.nc * d.G * d.Q * d.Q);
+    if (cb_int8) SSD_STAGE("chunk_bmm", launch_chunk_bmm_i8(d, Bq, Cq, cb8, s_cb, dbg ? &dd : nullptr, status, stream));
     if (tensor_core_shape(d))
         SSD_STAGE("chunk_scan", launch_chunk_scan_tc(d, true, x, Bq, Cq, Acs, dtc, D, sc, H8, y, dbg ? &dd : nullptr,
-                                                     scan_heads_per_cta(d), status, stream));
+                                                     scan_heads_per_cta(d), status, stream, cb_int8 ? cb8 : nullptr,
+                                                     s_cb, acs_half));
     else
         SSD_STAGE("chunk_scan", launch_chunk_scan_i8(d, x, dt, Acs, Bq, Cq, D, sc, H8, y, dbg ? &dd : nullptr, stream));
     if (dbg) {
         const size_t chains = (size_t)d.B * d.H;
         const size_t states = (size_t)d.B * d.nc * d.H * d.P * d.N;
-        if (dbg->Acs) SSD_TRY(cudaMemcpyAsync(dbg->Acs, Acs, chains * d.nc * d.Q * 4, cudaMemcpyDeviceToDevice, stream));
+        if (dbg->Acs && acs_half) SSD_TRY(launch_half_to_float(Acs, dbg->Acs, (long long)(chains * d.nc * d.Q), stream));
+        else if (dbg->Acs)
+            SSD_TRY(cudaMemcpyAsync(dbg->Acs, Acs, chains * d.nc * d.Q * 4, cudaMemcpyDeviceToDevice, stream));
         if (dbg->dq) SSD_TRY(cudaMemcpyAsync(dbg->dq, dq, chains * d.nc * 4, cudaMemcpyDeviceToDevice, stream));
         if (dbg->H8) SSD_TRY(cudaMemcpyAsync(dbg->H8, H8, states, cudaMemcpyDeviceToDevice, stream));
     }

@@ -34,6 +34,8 @@
 //               not coalesce).
 // Every wait is bounded; an expired wait raises a shared abort flag that ends all
 // roles, records SSD_ERR_TIMEOUT in the status word, and the CTA frees TMEM.
+#include <cuda_fp16.h>
+
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -54,7 +56,10 @@ constexpr int kRing = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 enum : uint32_t { kIdBuild = 1, kIdScale = 2, kIdStore = 3 };
 
-template <int Q, bool kI8>
+// kCB8 (W8A8, Q = 256; the notes' storage variant): ChunkScan2 reads CB as the INT8
+// codes ChunkBMM wrote to HBM (one step per tile) instead of forming CB on chip; the
+// B tile's space holds those codes and no ChunkBMM runs here.
+template <int Q, bool kI8, bool kCB8 = false>
 struct Cfg {
     static constexpr int JT = Q >= 128 ? Q / 128 : 1;            // 128-row tiles of the chunk
     static constexpr int CROWS = Q >= 128 ? Q : 128;             // C rows loaded (Q = 64: ghost rows)
@@ -67,7 +72,7 @@ struct Cfg {
     static constexpr uint32_t CBF = 128, CBP0 = 128, CBP1 = 0, RING = 192, YCOL = 256, TMEM_COLS = 512;
     static constexpr int EB = kI8 ? 1 : 2;
     static constexpr int C_BYTES = CROWS * kN * EB;
-    static constexpr int B_BYTES = Q * kN * EB;
+    static constexpr int B_BYTES = kCB8 ? Q * Q : Q * kN * EB;
     static constexpr int H_BYTES = kP * kN * EB;
     static constexpr int NHB = kI8 ? 2 : 1;                      // state tile buffers
     static constexpr int X_BYTES = Q * 128;
@@ -177,14 +182,28 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int Q, bool kI8>
+// Sixteen INT8 codes (one 16-byte word, first code in the lowest byte) as eight bf16
+// pairs: each code is exact in fp32 and in bf16 (at most 8 significant bits), so the
+// bf16 bits are the upper half of the fp32 bits.
+__device__ __forceinline__ void i8x16_to_bf16x8(const uint4 q, uint32_t (&o)[8]) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const uint32_t word = w[e >> 1] >> (16 * (e & 1));
+        const float lo = (float)(int)(int8_t)(word & 0xffu), hi = (float)(int)(int8_t)((word >> 8) & 0xffu);
+        o[e] = __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x7632);
+    }
+}
+
+template <int Q, bool kI8, bool kCB8>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_h,
                      const __grid_constant__ CUtensorMap tm_y, Dims d, int heads_per_cta, int ctas_per_group,
                      const float* __restrict__ Acs, const float* __restrict__ dtc, const float* __restrict__ Dv,
-                     I8Scales sc, I8Debug dbg, int* __restrict__ status) {
-    using K = Cfg<Q, kI8>;
+                     I8Scales sc, I8Debug dbg, int* __restrict__ status, const float* __restrict__ s_cb,
+                     int acs_half) {
+    using K = Cfg<Q, kI8, kCB8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -197,7 +216,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + K::OFF_TMEM);
     const long long vec_row0 = (((long long)b * d.H) * d.nc + c) * Q;   // + h * nc * Q
     const long long hc_row0 = ((long long)b * d.nc + c) * d.H;           // state rows (hc_row0 + h) * 64
-    const float sCB = kI8 ? __fmul_rn(__ldg(sc.s_C + g), __ldg(sc.s_B + g)) : 1.f;
+    float sCB = kI8 ? __fmul_rn(__ldg(sc.s_C + g), __ldg(sc.s_B + g)) : 1.f;
+    if (kCB8) sCB = __fmul_rn(sCB, __ldg(s_cb + ((long long)b * d.nc + c) * d.G + g));   // the CB codes' step
 
     if (tid == 0) {
         for (int i = 0; i < K::NBAR; ++i) {
@@ -241,17 +261,25 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                 tc::tma_load_3d(sm + K::OFF_C + K::CROWS * 128, &tm_c, bar + K::B_LOAD, g * kN + 64, c * Q, b);
                 tc::tma_load_3d(sm + K::OFF_B, &tm_b, bar + K::B_LOAD, g * kN, c * Q, b);
                 tc::tma_load_3d(sm + K::OFF_B + Q * 128, &tm_b, bar + K::B_LOAD, g * kN + 64, c * Q, b);
-            } else {
+            } else if (!kCB8) {
                 tc::tma_load_3d(sm + K::OFF_C, &tm_c, bar + K::B_LOAD, g * kN, c * Q, b);
                 tc::tma_load_3d(sm + K::OFF_B, &tm_b, bar + K::B_LOAD, g * kN, c * Q, b);
+            } else {
+                // the (b, c, g) CB codes as two 128-column halves, 128-byte swizzle
+                const int crow = (int)((((long long)b * d.nc + c) * d.G + g) * Q);
+                tc::tma_load_3d(sm + K::OFF_C, &tm_c, bar + K::B_LOAD, g * kN, c * Q, b);
+                tc::tma_load_2d(sm + K::OFF_B, &tm_b, bar + K::B_LOAD, 0, crow);
+                tc::tma_load_2d(sm + K::OFF_B + Q * 128, &tm_b, bar + K::B_LOAD, 128, crow);
             }
             for (int it = 0; it < nh; ++it) {
                 const int h = h0 + it, s = it & 1;
                 const uint32_t u = (uint32_t)(it >> 1);
                 if (!wait_bar<kI8>(bar + K::B_VEMPTY + s, (u & 1) ^ 1, abort_flag, status)) break;
-                tc::mbar_arrive_expect_tx(bar + K::B_VFULL + s, 2 * Q * 4);
+                const int acs_bytes = acs_half ? Q * 2 : Q * 4;
+                tc::mbar_arrive_expect_tx(bar + K::B_VFULL + s, acs_bytes + Q * 4);
                 const long long vr = vec_row0 + (long long)h * d.nc * Q;
-                tc::bulk_load(vec(s, kAcs), Acs + vr, Q * 4, bar + K::B_VFULL + s);
+                tc::bulk_load(vec(s, kAcs), reinterpret_cast<const uint8_t*>(Acs) + vr * (acs_half ? 2 : 4), acs_bytes,
+                              bar + K::B_VFULL + s);
                 tc::bulk_load(vec(s, kDtc), dtc + vr, Q * 4, bar + K::B_VFULL + s);
                 const int hb = kI8 ? s : 0;
                 const uint32_t hpar = kI8 ? ((u & 1) ^ 1) : (((uint32_t)it & 1) ^ 1);
@@ -291,7 +319,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             return __all_sync(0xffffffffu, tc::mbar_test(bar + which, parity));
         };
         bool ok = wait_all(K::B_LOAD, 0);
-        if (ok) {
+        if (ok && kCB8) {
+            // the CB codes are in shared memory: no ChunkBMM here
+            if (tc::elect_one()) tc::mbar_arrive(bar + K::B_CB);
+            __syncwarp();
+            ok = wait_all(K::B_PACKED, 0);
+        } else if (ok) {
             tc::tc_fence_after();
             if (tc::elect_one()) {
                 const uint32_t id0 = kI8 ? tc::idesc_s8_s32(128, K::NCB0, tc::kMajorK, tc::kMajorK)
@@ -401,7 +434,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
         bool ok = tc::named_and(kIdBuild, kBuilderThreads, wait_bar<kI8>(bar + K::B_CB, 0, abort_flag, status));
         tc::tc_fence_after();
-        if (ok && set == 0) {
+        if (ok && set == 0 && !kCB8) {
             if (kI8 && dbg.cb && (blockIdx.x % ctas_per_group) == 0) {
                 for (int J = 0; J < K::JT; ++J) {
                     const int ncol = J == 0 ? K::NCB0 : 256;
@@ -423,7 +456,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             // pack CB to bf16 pairs: tile 0 by set 0, tile 1 by set 1 (both in parallel;
             // the destinations do not overlap the other set's source columns)
             const int J = set;
-            if (J < K::JT) {
+            if (J < K::JT && !kCB8) {
                 const int ncol = J == 0 ? K::NCB0 : 256;
                 for (int g32 = 0; g32 < ncol / 32; ++g32) {
                     uint32_t v[32], w[16];
@@ -513,18 +546,40 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     for (int e = 0; e < 8; ++e) out[e] = 0u;
                 }
             };
+            // kCB8: the piece's two 16-code groups of row J*128 + rrow from the swizzled tile
+            auto cb8_load = [&](int k, uint32_t (&o0)[8], uint32_t (&o1)[8]) {
+                int J, ib;
+                piece_of(Q, k, J, ib);
+                const int row = J * 128 + rrow;
+#pragma unroll
+                for (int blk = 0; blk < 2; ++blk) {
+                    const int col = 32 * (2 * ib + blk) + c0;
+                    const int phys = ((col & 127) >> 4) ^ (row & 7);
+                    const uint4 q = *reinterpret_cast<const uint4*>(sm + K::OFF_B + (col >> 7) * (Q * 128) + row * 128 +
+                                                                    phys * 16);
+                    i8x16_to_bf16x8(q, blk == 0 ? o0 : o1);
+                }
+            };
             uint32_t cbv[2][2][8];                                // [buffer][block of the piece][packed cols]
-            tc::tmem_ld8(cb_cols(0), cbv[0][0]);
-            tc::tmem_ld8(cb_cols(0) + 16, cbv[0][1]);
-            tc::tmem_wait_ld();
+            if constexpr (kCB8) {
+                cb8_load(0, cbv[0][0], cbv[0][1]);
+            } else {
+                tc::tmem_ld8(cb_cols(0), cbv[0][0]);
+                tc::tmem_ld8(cb_cols(0) + 16, cbv[0][1]);
+                tc::tmem_wait_ld();
+            }
 #pragma unroll
             for (int k = 0; k < K::NPIECE; ++k) {
                 int J, ib;
                 piece_of(Q, k, J, ib);
                 const bool pre = k + 1 < K::NPIECE;
                 if (pre) {
-                    tc::tmem_ld8(cb_cols(k + 1), cbv[(k + 1) & 1][0]);
-                    tc::tmem_ld8(cb_cols(k + 1) + 16, cbv[(k + 1) & 1][1]);
+                    if constexpr (kCB8) {
+                        cb8_load(k + 1, cbv[(k + 1) & 1][0], cbv[(k + 1) & 1][1]);
+                    } else {
+                        tc::tmem_ld8(cb_cols(k + 1), cbv[(k + 1) & 1][0]);
+                        tc::tmem_ld8(cb_cols(k + 1) + 16, cbv[(k + 1) & 1][1]);
+                    }
                 }
                 const int pp = p + k, slot = pp % kRing;
                 const int jrow = J * 128 + rrow;                  // row of M (ghost rows >= Q when Q = 64)
@@ -578,10 +633,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     const int p = tid - kScaleWarp0 * 32;
                     vec(s, kMul)[p] = __ldg(sc.s_C + g) * __ldg(sc.s_s + h * kP + p);
                 }
+                const __half* acs_h = reinterpret_cast<const __half*>(acs);   // Acs stored as half
                 for (int i = tid - kScaleWarp0 * 32; i < Q; i += kEpiThreads) {
                     // explicitly rounded steps (no contraction), as in the single-launch scan
-                    const float ai = __fmul_rn(acs[i], kLog2e);
-                    const float ar = __fmul_rn(acs[i | 31], kLog2e);
+                    const float acs_i = acs_half ? __half2float(acs_h[i]) : acs[i];
+                    const float acs_r = acs_half ? __half2float(acs_h[i | 31]) : acs[i | 31];
+                    const float ai = __fmul_rn(acs_i, kLog2e);
+                    const float ar = __fmul_rn(acs_r, kLog2e);
                     const float dw = __fmul_rn(dts[i], sCB);
                     a2[i] = ai;
                     dtw[i] = __fsub_rn(lg2(dw), ai);              // log2(dt_i) - a_i; -inf when dt_i = 0
@@ -596,11 +654,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             if (!(ok = tc::named_and(kIdScale, kEpiThreads, wait_bar<kI8>(bar + K::B_YOFULL + s, u & 1, abort_flag, status))))
                 break;
             tc::tc_fence_after();
-            const float* acs = vec(s, kAcs);
+            const float* a2v = vec(s, kA2);                        // log2e * Acs, formed above
             const uint32_t ybase = trow + K::YCOL + 128 * s;
             for (int J = 0; J < K::JT; ++J) {
                 const int j = J * 128 + r;
-                const float e = ex2(fminf(__fmul_rn(acs[j < Q ? j : Q - 1], kLog2e), 0.f));
+                const float e = ex2(fminf(a2v[j < Q ? j : Q - 1], 0.f));
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     uint32_t v[32];
@@ -703,17 +761,20 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
     if (warp == 1) tc::tmem_dealloc(tmem, K::TMEM_COLS);
 }
 
-template <int Q, bool kI8>
+template <int Q, bool kI8, bool kCB8 = false>
 cudaError_t launch_q(const Dims& d, const CUtensorMap* maps, int hpc, int cpg, const float* Acs, const float* dtc,
-                     const float* D, const I8Scales& sc, const I8Debug* dbg, int* status, cudaStream_t st) {
-    using K = Cfg<Q, kI8>;
-    auto k = chunk_scan_tc_kernel<Q, kI8>;
+                     const float* D, const I8Scales& sc, const I8Debug* dbg, int* status, cudaStream_t st,
+                     const float* s_cb = nullptr, bool acs_half = false) {
+    using K = Cfg<Q, kI8, kCB8>;
+    static_assert(K::BYTES + 1024 <= 232448, "shared memory");
+    auto k = chunk_scan_tc_kernel<Q, kI8, kCB8>;
     const int smem = K::BYTES + 1024;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     I8Debug none{};
     k<<<dim3(d.G * cpg, d.nc, d.B), kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], d, hpc, cpg,
-                                                            Acs, dtc, D, sc, dbg ? *dbg : none, status);
+                                                            Acs, dtc, D, sc, dbg ? *dbg : none, status, s_cb,
+                                                            acs_half ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -722,9 +783,11 @@ cudaError_t launch_q(const Dims& d, const CUtensorMap* maps, int hpc, int cpg, c
 cudaError_t launch_chunk_scan_tc(const Dims& d, bool i8, const uint16_t* x, const void* Bmat,
                                  const void* Cmat, const float* Acs, const float* dtc, const float* D,
                                  const I8Scales& sc, const void* Hc, uint16_t* y, const I8Debug* dbg,
-                                 int heads_per_cta, int* status, cudaStream_t st) {
+                                 int heads_per_cta, int* status, cudaStream_t st, const int8_t* cb8,
+                                 const float* s_cb, bool acs_half) {
     if (d.B == 0 || d.nc == 0) return cudaSuccess;
     if (d.P != kP || d.N != kN) return cudaErrorInvalidValue;
+    if ((cb8 || acs_half) && (!i8 || d.Q != 256)) return cudaErrorInvalidValue;
     const int hpc = heads_per_cta < 1 ? 1 : (heads_per_cta > d.hpg ? d.hpg : heads_per_cta);
     const int cpg = (d.hpg + hpc - 1) / hpc;
     CUtensorMap maps[5];
@@ -747,7 +810,12 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, bool i8, const uint16_t* x, cons
     }
     ok = ok && make_tmap_3d(&maps[4], false, y, HP, d.L, d.B, HP * 2, d.Ls * HP * 2, 64, d.Q,
                             CU_TENSOR_MAP_SWIZZLE_128B);
+    if (cb8)   // the CB codes, [B * nc * G * Q rows][Q] int8, in 128-column halves
+        ok = ok && make_tmap_2d(&maps[1], true, cb8, d.Q, (unsigned long long)d.B * d.nc * d.G * d.Q, d.Q, 128, d.Q,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
+    if (cb8) return launch_q<256, true, true>(d, maps, hpc, cpg, Acs, dtc, D, sc, dbg, status, st, s_cb, acs_half);
+    if (acs_half) return launch_q<256, true>(d, maps, hpc, cpg, Acs, dtc, D, sc, dbg, status, st, nullptr, true);
     switch (d.Q) {
         case 64: return i8 ? launch_q<64, true>(d, maps, hpc, cpg, Acs, dtc, D, sc, dbg, status, st)
                            : launch_q<64, false>(d, maps, hpc, cpg, Acs, dtc, D, sc, dbg, status, st);

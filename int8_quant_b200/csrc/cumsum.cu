@@ -4,6 +4,9 @@
 // LUT_state[b,h,c,j] = dt_j * exp(Acs[Q-1] - Acs[j]) (eq. 4; the W8A8 path uses the
 // specified fp32 exp so that X_scaled's codes are reproducible) and dt in the same
 // chunk-major layout, so that the tensor-core kernels read both contiguously.
+// With `acs_half` (the notes' storage variant: dAcs kept in FP16) every Acs is rounded
+// to IEEE half (nearest even) as soon as it is formed, LUT_state and the decay code are
+// computed from the rounded values, and Acs is stored as half.
 //
 // One CTA per (chunk, block of 8 heads, batch row); warp k scans head h0 + k.  The
 // dt rows of the chunk are staged in shared memory (32-byte row segments, 8 heads x
@@ -14,6 +17,8 @@
 // order, so the result (and the W8A8 codes derived from it) is reproducible bit for
 // bit.  The results go back through shared memory so that every global store of a
 // warp covers 128 contiguous bytes.
+#include <cuda_fp16.h>
+
 #include "kernels.h"
 
 namespace ssd {
@@ -32,7 +37,7 @@ __global__ void __launch_bounds__(kThreads)
 cumsum_kernel(Dims d, const float* __restrict__ dt, const float* __restrict__ A,
               float* __restrict__ Acs, float* __restrict__ decay, int32_t* __restrict__ dq,
               int shift, int* __restrict__ status, float* __restrict__ lut, float* __restrict__ dtc,
-              I8Scales sc, float* __restrict__ inv_sx, float* __restrict__ mq) {
+              I8Scales sc, float* __restrict__ inv_sx, float* __restrict__ mq, int acs_half) {
     // this call's kernels record device-side errors in the workspace status word
     if (status && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) *status = kStatusOk;
     // W8A8: per-(h,p) quantisation reciprocal 1/s_x and requantisation multiplier
@@ -101,6 +106,7 @@ cumsum_kernel(Dims d, const float* __restrict__ dt, const float* __restrict__ A,
     for (int i = 0; i < 8; ++i) {
         if (i < m) {
             last = __fadd_rn(e, s[i]);
+            if (acs_half) last = __half2float(__float2half_rn(last));
             acsk[pad(lane * m + i)] = last;
         }
     }
@@ -112,7 +118,8 @@ cumsum_kernel(Dims d, const float* __restrict__ dt, const float* __restrict__ A,
         if (i < m) {
             const int j = lane + 32 * i;
             const float a = acsk[pad(j)];
-            Acs[row + j] = a;
+            if (acs_half) reinterpret_cast<__half*>(Acs)[row + j] = __float2half_rn(a);
+            else Acs[row + j] = a;
             if (lut) {
                 const float dtv = dtk[pad(j)];
                 lut[row + j] = kI8 ? __fmul_rn(dtv, ssd_expf(__fsub_rn(last, a))) : dtv * expf(last - a);
@@ -130,22 +137,37 @@ cumsum_kernel(Dims d, const float* __restrict__ dt, const float* __restrict__ A,
     }
 }
 
+// Half-precision values as fp32 (debug copies of a half Acs).
+__global__ void half_to_float_kernel(const __half* __restrict__ src, float* __restrict__ dst, long long n) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        dst[i] = __half2float(src[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_half_to_float(const void* src, float* dst, long long n, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const long long blocks = (n + 255) / 256;
+    half_to_float_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(static_cast<const __half*>(src),
+                                                                                   dst, n);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_cumsum(const Dims& d, const float* dt, const float* A, float* Acs,
                           float* decay, int32_t* dq, int shift, int* status, float* lut, float* dtc,
-                          cudaStream_t st, const I8Scales* sc, float* inv_sx, float* mq) {
+                          cudaStream_t st, const I8Scales* sc, float* inv_sx, float* mq, bool acs_half) {
     if (d.B == 0 || d.nc == 0) return cudaSuccess;
     dim3 grid(d.nc, (d.H + kHeadsPerCta - 1) / kHeadsPerCta, d.B);
     const size_t smem = (size_t)2 * kHeadsPerCta * (d.Q + d.Q / 32) * sizeof(float);
     if (dq) {
         cudaFuncSetAttribute(cumsum_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         cumsum_kernel<true><<<grid, kThreads, smem, st>>>(d, dt, A, Acs, decay, dq, shift, status, lut, dtc,
-                                                          sc ? *sc : I8Scales{}, sc ? inv_sx : nullptr, mq);
+                                                          sc ? *sc : I8Scales{}, sc ? inv_sx : nullptr, mq,
+                                                          acs_half ? 1 : 0);
     } else {
         cudaFuncSetAttribute(cumsum_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         cumsum_kernel<false><<<grid, kThreads, smem, st>>>(d, dt, A, Acs, decay, dq, shift, status, lut, dtc,
-                                                           I8Scales{}, nullptr, nullptr);
+                                                           I8Scales{}, nullptr, nullptr, 0);
     }
     return cudaGetLastError();
 }

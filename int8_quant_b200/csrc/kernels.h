@@ -12,7 +12,7 @@ namespace ssd {
 
 // Workspace layout of one scan call (offsets in bytes, 256-byte aligned regions).
 struct WsLayout {
-    size_t status, acs, lut, dtc, decay, states, passed, scales, total;
+    size_t status, acs, lut, dtc, decay, states, passed, scales, cb8, total;
 };
 // `fp32_states`: chunk states kept in fp32 (calibration) instead of bf16 / int8.
 WsLayout ws_layout(const Dims& d, bool i8, bool fp32_states = false);
@@ -27,6 +27,8 @@ struct I8Debug {
     int8_t* H8;
     int32_t* cb;
     int32_t* acc_scan1;
+    int8_t* cb8;      // storage variant: CB codes [B,nc,G,Q,Q]
+    double* s_cb;     // storage variant: their steps [B,nc,G]
 };
 
 struct I8Scales {
@@ -46,11 +48,14 @@ cudaError_t launch_quantize_bc(const Dims& d, const uint16_t* B, const uint16_t*
 // exp(Acs[Q-1]) (fp32 [B,H,nc]); the W8A8 path the decay codes (int32 [B,H,nc]).
 // Clears the workspace status word `status` (may be null) for the call.  `lut`
 // (LUT_state) and `dtc` (dt) are optional [B,H,nc,Q] outputs.  W8A8 with `sc`: also
-// inv_sx = 1/s_x and mq = s_x s_B / s_s per (h,p) ([H*P] each).
+// inv_sx = 1/s_x and mq = s_x s_B / s_s per (h,p) ([H*P] each).  `acs_half`: Acs rounded
+// to IEEE half as soon as it is formed, and stored as half (the storage variant).
 cudaError_t launch_cumsum(const Dims& d, const float* dt, const float* A, float* Acs,
                           float* decay, int32_t* dq, int shift, int* status, float* lut, float* dtc,
                           cudaStream_t st, const I8Scales* sc = nullptr, float* inv_sx = nullptr,
-                          float* mq = nullptr);
+                          float* mq = nullptr, bool acs_half = false);
+// n IEEE half values to fp32 (debug copies).
+cudaError_t launch_half_to_float(const void* src, float* dst, long long n, cudaStream_t st);
 
 // a2: ChunkState.  bf16: fp32 states [B,nc,H,P,N]; W8A8: INT8 states.
 // amax_xs / amax_s (calibration only): per-(h,p) running max of |X_scaled| and |S_c|.
@@ -112,7 +117,15 @@ bool make_tmap_2d(CUtensorMap* m, bool is_i8, const void* base, unsigned long lo
 cudaError_t launch_chunk_scan_tc(const Dims& d, bool i8, const uint16_t* x, const void* Bmat,
                                  const void* Cmat, const float* Acs, const float* dtc, const float* D,
                                  const I8Scales& sc, const void* Hc, uint16_t* y, const I8Debug* dbg,
-                                 int heads_per_cta, int* status, cudaStream_t st);
+                                 int heads_per_cta, int* status, cudaStream_t st, const int8_t* cb8 = nullptr,
+                                 const float* s_cb = nullptr, bool acs_half = false);
+
+// ChunkBMM of the notes' storage variant (W8A8, chunk 256, N = 128): per (b, c, g) the
+// INT32 CB tile, one fp64 step amax / 127, its INT8 codes to `cb8` [B,nc,G,Q,Q] and the
+// step as fp32 to `s_cb` [B,nc,G].  chunk_bmm_i8_bytes: workspace bytes of both.
+size_t chunk_bmm_i8_bytes(const Dims& d);
+cudaError_t launch_chunk_bmm_i8(const Dims& d, const int8_t* Bq, const int8_t* Cq, int8_t* cb8, float* s_cb,
+                                const I8Debug* dbg, int* status, cudaStream_t st);
 
 // Tensor-core ChunkState for P = 64, N = 128: one CTA per (head, chunk, batch row)
 // computes the chunk state transposed, S^T[n,p] = sum_j B[j,n] X_scaled[j,p], with

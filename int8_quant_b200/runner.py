@@ -63,13 +63,18 @@ class SsdProblem:
                                              initial_state, self.y, self.final32, self.ws_bf16, stream)
 
     # -- W8A8
-    def set_scales(self, s_B, s_C, s_x, s_s, shift: int = 7):
+    def set_scales(self, s_B, s_C, s_x, s_s, shift: int = 7, storage: int = 0):
+        """storage: 0, or SSD_STORAGE_* flags (the notes' storage variant)."""
         dev = self.inp["x"].device
         f = lambda a: torch.as_tensor(np.asarray(a, np.float32) if not torch.is_tensor(a) else a,
                                       dtype=torch.float32).to(dev).contiguous()
         self.scales = {"s_B": f(s_B), "s_C": f(s_C), "s_x": f(s_x), "s_s": f(s_s)}
         self.params = ssd.i8_params(self.scales["s_B"], self.scales["s_C"], self.scales["s_x"],
-                                    self.scales["s_s"], shift)
+                                    self.scales["s_s"], shift, storage)
+
+    def set_storage(self, storage: int):
+        """Switch the W8A8 calls between the library's layout (0) and the storage variant."""
+        self.params.storage = int(storage)
 
     def calibrate(self, prefix: int = 512, shift: int = 7, stream=None):
         b, L, H, P, G, N, Q = self.dims
@@ -116,6 +121,9 @@ class SsdProblem:
             "cb": torch.zeros((b, nc, G, Q, Q), dtype=torch.int32, device=dev),
             "acc_scan1": torch.zeros((b, Lp, H, P), dtype=torch.int32, device=dev),
         }
+        if self.params.storage & ssd.SSD_STORAGE_CB_INT8:
+            dbg["cb8"] = torch.zeros((b, nc, G, Q, Q), dtype=torch.int8, device=dev)
+            dbg["s_cb"] = torch.zeros((b, nc, G), dtype=torch.float64, device=dev)
         self.quantize(stream)
         i = self.inp
         ssd.ssd_scan_fwd_i8_debug(self.shape, i["x"], i["dt"], i["A"], self.Bq, self.Cq, i["D"], self.params,

@@ -45,11 +45,16 @@ class SsdShape(ctypes.Structure):
 
 class SsdI8Params(ctypes.Structure):
     _fields_ = [("s_B", ctypes.c_void_p), ("s_C", ctypes.c_void_p), ("s_x", ctypes.c_void_p),
-                ("s_s", ctypes.c_void_p), ("decay_shift", ctypes.c_int)]
+                ("s_s", ctypes.c_void_p), ("decay_shift", ctypes.c_int), ("storage", ctypes.c_int)]
+
+
+SSD_STORAGE_ACS_FP16 = 1
+SSD_STORAGE_CB_INT8 = 2
 
 
 class SsdI8Debug(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("Acs", "dq", "Xq", "acc_state", "S8", "H8", "cb", "acc_scan1")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("Acs", "dq", "Xq", "acc_state", "S8", "H8", "cb", "acc_scan1",
+                                               "cb8", "s_cb")]
 
 
 class SsdError(RuntimeError):
@@ -232,8 +237,9 @@ def ssd_static_scratch_status(stream=None) -> int:
     return int(_lib().ssd_static_scratch_status(_stream(stream)))
 
 
-def i8_params(s_B, s_C, s_x, s_s, decay_shift=7) -> SsdI8Params:
-    return SsdI8Params(s_B.data_ptr(), s_C.data_ptr(), s_x.data_ptr(), s_s.data_ptr(), int(decay_shift))
+def i8_params(s_B, s_C, s_x, s_s, decay_shift=7, storage=0) -> SsdI8Params:
+    return SsdI8Params(s_B.data_ptr(), s_C.data_ptr(), s_x.data_ptr(), s_s.data_ptr(), int(decay_shift),
+                       int(storage))
 
 
 def ssd_scan_fwd_i8(shape, x, dt, A, Bq, Cq, D, params: SsdI8Params, y, final_state, workspace, stream=None):

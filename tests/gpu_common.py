@@ -44,11 +44,12 @@ def oracle_scales(inp: dict, chunk: int, prefix: int = 512) -> dict:
                        prefix)
 
 
-def oracle_i8(inp: dict, sc: dict, chunk: int, shift: int = 7) -> dict:
+def oracle_i8(inp: dict, sc: dict, chunk: int, shift: int = 7, **variant) -> dict:
+    """The integer W8A8 oracle on the workload's inputs; `variant`: acs_fp16 / cb_int8 switches."""
     Bv, Cv = as_float(inp["B"]).astype(F32), as_float(inp["C"]).astype(F32)
     Bq, Cq = W.quantize_inputs(Bv, Cv, sc["s_B"], sc["s_C"])
     r = W.ssd_w8a8(as_float(inp["x"]).astype(F32), inp["dt"], inp["A"], Bq, Cq, inp["D"], sc["s_B"], sc["s_C"],
-                   sc["s_x"], sc["s_s"], chunk, shift)
+                   sc["s_x"], sc["s_s"], chunk, shift, **variant)
     r["Bq"], r["Cq"] = Bq, Cq
     return r
 
