@@ -8,6 +8,7 @@ namespace ssd {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kMaxGroups = 64;                     // groups whose 1/s a CTA keeps in shared memory
 
 __global__ void __launch_bounds__(kThreads)
 quantize_bc_kernel(const uint4* __restrict__ B, const uint4* __restrict__ C,
@@ -16,9 +17,15 @@ quantize_bc_kernel(const uint4* __restrict__ B, const uint4* __restrict__ C,
     const uint4* src = blockIdx.y == 0 ? B : C;
     uint2* dst = blockIdx.y == 0 ? Bq : Cq;
     const float* s = blockIdx.y == 0 ? s_B : s_C;
+    // IEEE 1/s per group, once per CTA
+    __shared__ float inv_s[kMaxGroups];
+    for (int g = threadIdx.x; g < G && g < kMaxGroups; g += kThreads) inv_s[g] = __frcp_rn(__ldg(s + g));
+    __syncthreads();
     const int vec_per_group = N / 8;
     const long long stride = (long long)gridDim.x * kThreads;
     constexpr int kUnroll = 4;                           // loads in flight per thread
+    const float2 lo = make_float2(-127.0f, -127.0f), hi = make_float2(127.0f, 127.0f);
+    const float2 rnd = make_float2(12582912.0f, 12582912.0f);   // 1.5 * 2^23
     for (long long i0 = blockIdx.x * (long long)kThreads + threadIdx.x; i0 < nvec; i0 += kUnroll * stride) {
         uint4 vv[kUnroll];
 #pragma unroll
@@ -31,17 +38,26 @@ quantize_bc_kernel(const uint4* __restrict__ B, const uint4* __restrict__ C,
             const long long i = i0 + r * stride;
             if (i >= nvec) break;
             const int g = (int)((i / vec_per_group) % G);
-            const float inv = __frcp_rn(__ldg(s + g));     // IEEE 1/s
+            const float inv = g < kMaxGroups ? inv_s[g] : __frcp_rn(__ldg(s + g));
+            const float2 inv2 = make_float2(inv, inv);
             const uint4 v = vv[r];
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t out[2] = {0u, 0u};
+            uint32_t b[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint16_t bits = (uint16_t)(w[k >> 1] >> ((k & 1) * 16));
-                const int q = quant_i8(bf16_bits_to_float(bits), inv);
-                out[k >> 2] |= ((uint32_t)(q & 0xff)) << ((k & 3) * 8);
+            for (int k = 0; k < 4; ++k) {
+                // clamp(rint(x / s), +-127): the product rounded in fp32, clamped (the same code:
+                // +-127 are integers), rounded to nearest even by adding 1.5 * 2^23, whose low
+                // byte is then the code's byte
+                float2 q = __fmul2_rn(make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u)),
+                                      inv2);
+                q.x = fminf(fmaxf(q.x, lo.x), hi.x);
+                q.y = fminf(fmaxf(q.y, lo.y), hi.y);
+                q = __fadd2_rn(q, rnd);
+                b[2 * k] = __float_as_uint(q.x);
+                b[2 * k + 1] = __float_as_uint(q.y);
             }
-            dst[i] = make_uint2(out[0], out[1]);
+            dst[i] = make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410),
+                                __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
         }
     }
 }

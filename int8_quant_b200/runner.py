@@ -132,9 +132,14 @@ class SsdProblem:
 
 
 class StreamedScan:
-    """A batch held in pinned host memory, scanned in groups of batch rows with the copies
-    overlapped: group g's host->device copy, group g-1's scan and group g-2's device->host
-    copy run on three streams at once (batch rows are independent problems).
+    """A batch held in pinned host memory, scanned in groups with the copies overlapped:
+    group g's host->device copy, group g-1's scan and group g-2's device->host copy run on
+    three streams at once.  A group is `rows_per_group` batch rows (independent problems)
+    or, with `seg_len`, one batch row's segment of seg_len tokens (a multiple of the chunk):
+    the segments of a row are scanned in order, each from the previous one's final state
+    (ssd_scan_fwd_*_from_state, which reproduces one call over the whole row bit for bit
+    when the splits fall on chunk boundaries), so that many small groups keep the copy
+    engines busy from the first group's copy to the last one's.
 
     host: pinned CPU tensors x [B,L,H,P] (bf16), dt [B,L,H], B and C [B,L,G,N] (bf16), and
     the outputs y [B,L,H,P] (bf16) and final [B,H,P,N] (fp32 for bf16, int8 for W8A8).
@@ -142,24 +147,33 @@ class StreamedScan:
     """
 
     def __init__(self, host: dict, A, D, chunk: int, path: str, rows_per_group: int = 1, scales=None,
-                 shift: int = 7, device="cuda"):
+                 shift: int = 7, device="cuda", seg_len: int | None = None):
         assert path in ("bf16", "w8a8")
         self.h, self.path, self.A, self.D = host, path, A, D
         b, L, H, P = host["x"].shape
         G, N = host["B"].shape[2], host["B"].shape[3]
-        self.rows = rows_per_group
-        self.groups = [(r, min(rows_per_group, b - r)) for r in range(0, b, rows_per_group)]
-        self.shape = ssd.SsdShape.of(rows_per_group, L, H, P, G, N, chunk)
+        seg = L if seg_len is None or seg_len >= L else int(seg_len)
+        if seg < L:
+            assert rows_per_group == 1 and seg % chunk == 0, "segments: one row per group, whole chunks"
+        self.rows, self.seg, self.L, self.chunk = rows_per_group, seg, L, chunk
+        # (first row, rows, first token, tokens)
+        self.groups = [(r, min(rows_per_group, b - r), t0, min(seg, L - t0))
+                       for r in range(0, b, rows_per_group) for t0 in range(0, max(L, 1), max(seg, 1))]
+        self.shape = ssd.SsdShape.of(rows_per_group, seg, H, P, G, N, chunk)
         dev = torch.device(device)
         i8 = path == "w8a8"
         self.slots = []
         for _ in range(2):
-            sl = {k: torch.empty((rows_per_group,) + tuple(host[k].shape[1:]), dtype=host[k].dtype, device=dev)
-                  for k in ("x", "dt", "B", "C", "y", "final")}
+            sl = {k: torch.empty((rows_per_group, seg) + tuple(host[k].shape[2:]), dtype=host[k].dtype, device=dev)
+                  for k in ("x", "dt", "B", "C", "y")}
+            sl["final"] = torch.empty((rows_per_group,) + tuple(host["final"].shape[1:]), dtype=host["final"].dtype,
+                                      device=dev)
             if i8:
                 sl["Bq"] = torch.empty(sl["B"].shape, dtype=torch.int8, device=dev)
                 sl["Cq"] = torch.empty(sl["C"].shape, dtype=torch.int8, device=dev)
             self.slots.append(sl)
+        # the state carried between the segments of a row (two buffers: read one, write the other)
+        self.carry = [torch.empty_like(self.slots[0]["final"]) for _ in range(2)]
         self.ws = torch.empty(max(ssd.ssd_workspace_bytes(self.shape, i8), 256), dtype=torch.uint8, device=dev)
         if i8:
             self.scales = scales
@@ -173,37 +187,44 @@ class StreamedScan:
     def run(self):
         """Enqueue the whole batch; returns at once (synchronise on `self.streams[2]`)."""
         s_in, s_cmp, s_out = self.streams
-        for r0, n in self.groups:
+        sh = self.shape
+        for r0, n, t0, ln in self.groups:
             g = self.seq
             self.seq += 1
             k = g % 2
             sl = self.slots[k]
-            shape = self.shape if n == self.rows else ssd.SsdShape.of(
-                n, self.shape.seqlen, self.shape.nheads, self.shape.headdim, self.shape.ngroups, self.shape.dstate,
-                self.shape.chunk)
+            first, last = t0 == 0, t0 + ln >= self.L
+            shape = sh if (n, ln) == (self.rows, self.seg) else ssd.SsdShape.of(
+                n, ln, sh.nheads, sh.headdim, sh.ngroups, sh.dstate, sh.chunk)
+            seg_i = t0 // self.seg
+            init = None if first else self.carry[(seg_i - 1) % 2][:n]
+            fin = sl["final"][:n] if last else self.carry[seg_i % 2][:n]
             with torch.cuda.stream(s_in):
                 if g >= 2:
                     s_in.wait_event(self.ev["done"][k])             # slot's inputs consumed by scan g-2
                 for name in ("x", "dt", "B", "C"):
-                    sl[name][:n].copy_(self.h[name][r0:r0 + n], non_blocking=True)
+                    sl[name][:n, :ln].copy_(self.h[name][r0:r0 + n, t0:t0 + ln], non_blocking=True)
                 self.ev["in"][k].record(s_in)
             with torch.cuda.stream(s_cmp):
                 s_cmp.wait_event(self.ev["in"][k])
                 if g >= 2:
                     s_cmp.wait_event(self.ev["out"][k])            # slot's outputs read by copy g-2
+                x, dt, y = sl["x"][:n, :ln], sl["dt"][:n, :ln], sl["y"][:n, :ln]
                 if self.path == "w8a8":
-                    ssd.ssd_quantize_inputs(shape, sl["B"], sl["C"], self.scales["s_B"], self.scales["s_C"], sl["Bq"],
-                                            sl["Cq"], s_cmp)
-                    ssd.ssd_scan_fwd_i8(shape, sl["x"], sl["dt"], self.A, sl["Bq"], sl["Cq"], self.D, self.params,
-                                        sl["y"], sl["final"], self.ws, s_cmp)
+                    Bq, Cq = sl["Bq"][:n, :ln], sl["Cq"][:n, :ln]
+                    ssd.ssd_quantize_inputs(shape, sl["B"][:n, :ln], sl["C"][:n, :ln], self.scales["s_B"],
+                                            self.scales["s_C"], Bq, Cq, s_cmp)
+                    ssd.ssd_scan_fwd_i8_from_state(shape, x, dt, self.A, Bq, Cq, self.D, self.params, init, y, fin,
+                                                   self.ws, s_cmp)
                 else:
-                    ssd.ssd_scan_fwd_bf16(shape, sl["x"], sl["dt"], self.A, sl["B"], sl["C"], self.D, sl["y"],
-                                          sl["final"], self.ws, s_cmp)
+                    ssd.ssd_scan_fwd_bf16_from_state(shape, x, dt, self.A, sl["B"][:n, :ln], sl["C"][:n, :ln],
+                                                     self.D, init, y, fin, self.ws, s_cmp)
                 self.ev["done"][k].record(s_cmp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(self.ev["done"][k])
-                self.h["y"][r0:r0 + n].copy_(sl["y"][:n], non_blocking=True)
-                self.h["final"][r0:r0 + n].copy_(sl["final"][:n], non_blocking=True)
+                self.h["y"][r0:r0 + n, t0:t0 + ln].copy_(sl["y"][:n, :ln], non_blocking=True)
+                if last:
+                    self.h["final"][r0:r0 + n].copy_(sl["final"][:n], non_blocking=True)
                 self.ev["out"][k].record(s_out)
 
 

@@ -154,6 +154,39 @@ def test_workspace_status_is_ok_after_a_run(torch_cuda):
 
 
 @pytest.mark.parametrize("path", ["bf16", "w8a8"])
+@pytest.mark.parametrize("name", ["ragged-q256", "ragged-q64"])
+def test_streamed_segments_equal_whole_batch(torch_cuda, name, path):
+    """Host-resident batch streamed one row's segment of 2 chunks at a time, each segment
+    continuing from the previous one's state (the last one ragged): y and the final
+    state equal the whole-batch call bit for bit."""
+    from int8_quant_b200.runner import StreamedScan
+    torch = torch_cuda
+    w = CASES[name].with_(batch=3)
+    inp, pb = _problem(torch_cuda, w)
+    if path == "w8a8":
+        sc = oracle_scales(inp, w.chunk, w.calib_prefix)
+        pb.set_scales(sc["s_B"], sc["s_C"], sc["s_x"], sc["s_s"], 7)
+        pb.run_i8()
+        fin = pb.final8
+    else:
+        pb.run_bf16()
+        fin = pb.final32
+    torch.cuda.synchronize()
+    host = {k: pb.inp[k].to("cpu").pin_memory() for k in ("x", "dt", "B", "C")}
+    host["y"] = torch.empty_like(pb.y, device="cpu").pin_memory()
+    host["final"] = torch.empty_like(fin, device="cpu").pin_memory()
+    run = StreamedScan(host, pb.inp["A"], pb.inp["D"], w.chunk, path, rows_per_group=1,
+                       scales=pb.scales if path == "w8a8" else None, seg_len=2 * w.chunk)
+    assert len(run.groups) == 3 * ((w.seqlen + 2 * w.chunk - 1) // (2 * w.chunk)) > 3
+    for _ in range(2):
+        host["y"].view(torch.int16).fill_(-1)
+        run.run()
+        torch.cuda.synchronize()
+        assert torch.equal(host["y"].view(torch.int16), pb.y.cpu().view(torch.int16))
+        assert torch.equal(host["final"], fin.cpu())
+
+
+@pytest.mark.parametrize("path", ["bf16", "w8a8"])
 @pytest.mark.parametrize("name", ["ragged-q256", "tiny-ragged"])
 def test_streamed_batch_equals_whole_batch(torch_cuda, name, path):
     """Host-resident batch run group by group with overlapped copies (two rows per group,
