@@ -64,7 +64,9 @@ struct StateCfg {
     static constexpr int OFF_BAR = OFF_SX + NS * SX_BYTES;
     static constexpr int OFF_FLAG = OFF_BAR + NBAR * 8;
     static constexpr int OFF_TMEM = OFF_FLAG + 8;
-    static constexpr int BYTES = OFF_TMEM + 8;
+    // W8A8: each epilogue warp's copy of its unit's 64 requantisation factors (16-byte aligned)
+    static constexpr int OFF_MQ = (OFF_TMEM + 8 + 15) & ~15;
+    static constexpr int BYTES = OFF_MQ + (kI8 ? 4 * kP * 4 : 0);
 };
 
 // INT8 code of an already scaled value, clamp(rint(v), +-127), without a conversion
@@ -288,6 +290,14 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                 m1 = __ldg(mq_g + h * kP + lane + 32);
             }
             const int t = k % kAcc;
+            // the unit's factors, broadcast to the warp through shared memory (16-byte reads)
+            float* mqw = reinterpret_cast<float*>(sm + K::OFF_MQ) + quarter * kP;
+            if (kI8) {
+                __syncwarp();                                          // the previous unit's reads are done
+                mqw[lane] = c0;
+                mqw[lane + 32] = c1;
+                __syncwarp();
+            }
             const bool ok = tc::wait_or_abort(bar + K::TFULL + t, (uint32_t)(k / kAcc) & 1, abort_flag, status,
                                               kStatusTimeout);
             if (!__all_sync(0xffffffffu, ok)) break;
@@ -309,8 +319,8 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
 #pragma unroll
                 for (int p = 0; p < kP; p += 2) {
                     const uint32_t a0 = p < 32 ? v0[p] : v1[p - 32], a1 = p < 32 ? v0[p + 1] : v1[p - 31];
-                    const float mq0 = __shfl_sync(0xffffffffu, p < 32 ? c0 : c1, p & 31);
-                    const float mq1 = __shfl_sync(0xffffffffu, p < 32 ? c0 : c1, (p + 1) & 31);
+                    const float2 mq2 = reinterpret_cast<const float2*>(mqw)[p >> 1];
+                    const float mq0 = mq2.x, mq1 = mq2.y;
                     float f0, f1, r0, r1;
                     // int-to-float conversions: they run on a pipe of their own, which is idle here
                     f0 = __int2float_rn((int)a0);
