@@ -133,8 +133,8 @@ class SsdProblem:
 
 class StreamedScan:
     """A batch held in pinned host memory, scanned in groups with the copies overlapped:
-    group g's host->device copy, group g-1's scan and group g-2's device->host copy run on
-    three streams at once.  A group is `rows_per_group` batch rows (independent problems)
+    host->device copies, scans and device->host copies run on three streams, groups taking
+    turns in `nslots` device buffers.  A group is `rows_per_group` batch rows (independent problems)
     or, with `seg_len`, one batch row's segment of seg_len tokens (a multiple of the chunk):
     the segments of a row are scanned in order, each from the previous one's final state
     (ssd_scan_fwd_*_from_state, which reproduces one call over the whole row bit for bit
@@ -147,7 +147,7 @@ class StreamedScan:
     """
 
     def __init__(self, host: dict, A, D, chunk: int, path: str, rows_per_group: int = 1, scales=None,
-                 shift: int = 7, device="cuda", seg_len: int | None = None):
+                 shift: int = 7, device="cuda", seg_len: int | None = None, nslots: int = 2):
         assert path in ("bf16", "w8a8")
         self.h, self.path, self.A, self.D = host, path, A, D
         b, L, H, P = host["x"].shape
@@ -162,8 +162,9 @@ class StreamedScan:
         self.shape = ssd.SsdShape.of(rows_per_group, seg, H, P, G, N, chunk)
         dev = torch.device(device)
         i8 = path == "w8a8"
+        self.nslots = max(2, int(nslots))
         self.slots = []
-        for _ in range(2):
+        for _ in range(self.nslots):
             sl = {k: torch.empty((rows_per_group, seg) + tuple(host[k].shape[2:]), dtype=host[k].dtype, device=dev)
                   for k in ("x", "dt", "B", "C", "y")}
             sl["final"] = torch.empty((rows_per_group,) + tuple(host["final"].shape[1:]), dtype=host["final"].dtype,
@@ -179,7 +180,7 @@ class StreamedScan:
             self.scales = scales
             self.params = ssd.i8_params(scales["s_B"], scales["s_C"], scales["s_x"], scales["s_s"], shift)
         self.streams = [torch.cuda.Stream(device=dev) for _ in range(3)]      # h2d, compute, d2h
-        self.ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "done", "out")}
+        self.ev = {k: [torch.cuda.Event() for _ in range(self.nslots)] for k in ("in", "done", "out")}
         self.seq = 0                                                           # groups enqueued so far
         self.h2d_bytes = sum(host[k].numel() * host[k].element_size() for k in ("x", "dt", "B", "C"))
         self.d2h_bytes = sum(host[k].numel() * host[k].element_size() for k in ("y", "final"))
@@ -191,7 +192,7 @@ class StreamedScan:
         for r0, n, t0, ln in self.groups:
             g = self.seq
             self.seq += 1
-            k = g % 2
+            k = g % self.nslots
             sl = self.slots[k]
             first, last = t0 == 0, t0 + ln >= self.L
             shape = sh if (n, ln) == (self.rows, self.seg) else ssd.SsdShape.of(
@@ -200,15 +201,15 @@ class StreamedScan:
             init = None if first else self.carry[(seg_i - 1) % 2][:n]
             fin = sl["final"][:n] if last else self.carry[seg_i % 2][:n]
             with torch.cuda.stream(s_in):
-                if g >= 2:
-                    s_in.wait_event(self.ev["done"][k])             # slot's inputs consumed by scan g-2
+                if g >= self.nslots:
+                    s_in.wait_event(self.ev["done"][k])             # slot's inputs consumed by its last scan
                 for name in ("x", "dt", "B", "C"):
                     sl[name][:n, :ln].copy_(self.h[name][r0:r0 + n, t0:t0 + ln], non_blocking=True)
                 self.ev["in"][k].record(s_in)
             with torch.cuda.stream(s_cmp):
                 s_cmp.wait_event(self.ev["in"][k])
-                if g >= 2:
-                    s_cmp.wait_event(self.ev["out"][k])            # slot's outputs read by copy g-2
+                if g >= self.nslots:
+                    s_cmp.wait_event(self.ev["out"][k])            # slot's outputs read by its last copy
                 x, dt, y = sl["x"][:n, :ln], sl["dt"][:n, :ln], sl["y"][:n, :ln]
                 if self.path == "w8a8":
                     Bq, Cq = sl["Bq"][:n, :ln], sl["Cq"][:n, :ln]
