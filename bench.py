@@ -442,7 +442,7 @@ def run_ours(args, rank, world, dist):
                 "kernel_shares": {k: round(v[0] / sum(x[0] for x in kern.values()), 4) for k, v in kern.items()}}
 
     def path_roofline(path, ms, w=w):
-        """The step against the benchmark spec's roofline: the slower of the compulsory HBM bytes over
+        """The step against the SSD scan's roofline: the slower of the compulsory HBM bytes over
         8 TB/s and the contractions at the datasheet tensor peaks (bf16 2.25 PFLOP/s, int8
         4.5 POP/s), and the same with this machine's measured peaks (copy bandwidth; bf16 GEMM,
         int8 taken as twice it)."""
