@@ -110,7 +110,9 @@ const char* ssd_last_cuda_error(void);
 /* Bytes of device workspace that ssd_scan_fwd_bf16 (is_i8 = 0) or ssd_scan_fwd_i8
  * (is_i8 = 1) need for `shape`; 0 for an invalid or unsupported shape.  The
  * workspace holds the per-chunk cumulative decays, chunk states and passed states
- * plus a device status word; its contents are private to the library. */
+ * plus a device status word (W8A8: also room for the single-launch scan's flags and
+ * the storage variant's CB codes, so one size serves every W8A8 mode); its contents
+ * are private to the library. */
 size_t ssd_workspace_bytes(const ssd_shape* shape, int is_i8);
 
 /* ChunkBMM/ChunkScan inputs quantised once along G ("SSDi8" notes, key design 3):

@@ -85,6 +85,15 @@ def test_invalid_arguments_fail_before_any_launch():
     assert lib.ssd_scan_fwd_i8(ctypes.byref(s), f, f, f, f, f, f, ctypes.byref(p), f, f, f, wsi, None) == 1
     p.decay_shift = 15
     assert lib.ssd_scan_fwd_i8(ctypes.byref(s), f, f, f, f, f, f, ctypes.byref(p), f, f, f, wsi, None) == 1
+    # the storage variant: unknown flags; a chunk other than 256 or the (16, 16) shape is unsupported
+    p.decay_shift = 7
+    p.storage = 4
+    assert lib.ssd_scan_fwd_i8(ctypes.byref(s), f, f, f, f, f, f, ctypes.byref(p), f, f, f, wsi, None) == 1
+    p.storage = iq.SSD_STORAGE_ACS_FP16 | iq.SSD_STORAGE_CB_INT8
+    s128 = iq.SsdShape.of(1, 256, 4, 64, 1, 128, 128)
+    assert lib.ssd_scan_fwd_i8(ctypes.byref(s128), f, f, f, f, f, f, ctypes.byref(p), f, f, f, 1 << 30, None) == 2
+    s16 = iq.SsdShape.of(1, 256, 4, 16, 1, 16, 256)
+    assert lib.ssd_scan_fwd_i8(ctypes.byref(s16), f, f, f, f, f, f, ctypes.byref(p), f, f, f, 1 << 30, None) == 2
     # quantize: null outputs
     assert lib.ssd_quantize_inputs(ctypes.byref(s), f, f, f, f, None, f, None) == 1
     # calibration: workspace too small
