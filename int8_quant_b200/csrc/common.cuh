@@ -78,6 +78,24 @@ __device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
     return r;
 }
 
+// One link of the integer StatePassing (eq. 6) on four codes per word, for decay shifts
+// k <= 7 and decay codes dq <= 2^k: H' = sat127(S8 + ((dq H + 2^(k-1)) >> k)).  With
+// Hu = H + 128 and Su = S8 + 128 (the codes with the top bit flipped),
+// V = dq Hu + 2^(k-1) + 128 (2^k - dq) + Su 2^k = dq H + 2^(k-1) + (S8 + 256) 2^k lies in
+// [0, 2^16), so two codes share a 32-bit word as 16-bit fields; V >> k = H' + 256 before
+// saturation, so clamping V to [129 2^k, 384 2^k - 1] (lo, hi: both fields) saturates, and
+// the low byte of each field of V >> k is H' as an int8 code (bits shifted down from the
+// upper field land at bit 16 - k >= 9, above it).  k0 = 2^(k-1) + 128 (2^k - dq) in both
+// fields.
+__device__ __forceinline__ uint32_t chain_word(uint32_t h4, uint32_t s4, uint32_t dq, uint32_t k0, int k,
+                                               uint32_t lo, uint32_t hi) {
+    const uint32_t hu = h4 ^ 0x80808080u, su = s4 ^ 0x80808080u;
+    uint32_t v0 = __byte_perm(hu, 0, 0x4140) * dq + k0 + (__byte_perm(su, 0, 0x4140) << k);
+    uint32_t v1 = __byte_perm(hu, 0, 0x4342) * dq + k0 + (__byte_perm(su, 0, 0x4342) << k);
+    v0 = min_u16x2(max_u16x2(v0, lo), hi) >> k;
+    v1 = min_u16x2(max_u16x2(v1, lo), hi) >> k;
+    return __byte_perm(v0, v1, 0x6420);
+}
 // atomicMax on non-negative floats through their (monotone) bit patterns.
 __device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
     atomicMax(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));

@@ -285,22 +285,6 @@ __device__ __noinline__ int poll_flag(const int* f, int want, volatile int* abor
     }
 }
 
-// One link of the integer StatePassing on four codes per word, for decay shifts k <= 7:
-// H' = sat127(S8 + ((dq H + 2^(k-1)) >> k)).  With Hu = H + 128 and Su = S8 + 128 (the
-// codes with the top bit flipped), V = dq Hu + 2^(k-1) + 128 (2^k - dq) + Su 2^k
-// = dq H + 2^(k-1) + (S8 + 256) 2^k lies in [2^(k+1), 510 2^k + 2^(k-1)] < 2^16, so two
-// codes share a 32-bit word as 16-bit fields; V >> k = H' + 256 before saturation, so
-// clamping V to [129 2^k, 384 2^k - 1] saturates, and the low byte of V >> k is H' as
-// an int8 code.
-__device__ __forceinline__ uint32_t chain_word(uint32_t h4, uint32_t s4, uint32_t dq, uint32_t k0, int k,
-                                               uint32_t lo, uint32_t hi) {
-    const uint32_t hu = h4 ^ 0x80808080u, su = s4 ^ 0x80808080u;
-    uint32_t v0 = __byte_perm(hu, 0, 0x4140) * dq + k0 + (__byte_perm(su, 0, 0x4140) << k);
-    uint32_t v1 = __byte_perm(hu, 0, 0x4342) * dq + k0 + (__byte_perm(su, 0, 0x4342) << k);
-    v0 = min_u16x2(max_u16x2(v0, lo), hi) >> k;
-    v1 = min_u16x2(max_u16x2(v1, lo), hi) >> k;
-    return __byte_perm(v0, v1, 0x6420);
-}
 // The same link, one code at a time (any k): w holds S8 (in) and H_{c+1} (out) for the
 // 64 codes of row n; hrow is H_c's row (64 bytes).
 __device__ __noinline__ void chain_row_generic(uint32_t* w, const uint32_t* hrow, int dq, int k) {

@@ -93,24 +93,10 @@ state_passing_i8_kernel(Dims d, const int8_t* __restrict__ S8, const int32_t* __
     const int8_t* s = S8 + ((long long)b * d.nc * d.H + h) * PN + e;
     int8_t* hc = H8 + ((long long)b * d.nc * d.H + h) * PN + e;
     const int32_t* q = dq + ((long long)b * d.H + h) * d.nc;
-    const int half = 1 << (shift - 1);
-    int hv[kVecI8];
-#pragma unroll
-    for (int v = 0; v < kVecI8; ++v) hv[v] = 0;
-    if (init8) {
-        const uint4 t = __ldg(reinterpret_cast<const uint4*>(init8 + ((long long)b * d.H + h) * PN + e));
-        const uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-        for (int v = 0; v < kVecI8; ++v) hv[v] = (int)(int8_t)(w[v >> 2] >> (8 * (v & 3)));
-    }
-    auto pack = [&]() -> uint4 {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            w[i] = __byte_perm(__byte_perm(hv[4 * i], hv[4 * i + 1], 0x0040), __byte_perm(hv[4 * i + 2], hv[4 * i + 3], 0x0040),
-                               0x5410);
-        return make_uint4(w[0], w[1], w[2], w[3]);
-    };
+    // the state: 16 codes, four to a word (first code in the lowest byte)
+    uint4 hw = init8 ? __ldg(reinterpret_cast<const uint4*>(init8 + ((long long)b * d.H + h) * PN + e))
+                     : make_uint4(0, 0, 0, 0);
+    const uint32_t lo = (129u << shift) * 0x10001u, hi = ((384u << shift) - 1u) * 0x10001u;
     constexpr int kAheadI8 = 4;
     for (int c0 = 0; c0 < d.nc; c0 += kAheadI8) {
         uint4 sv[kAheadI8];
@@ -125,17 +111,31 @@ state_passing_i8_kernel(Dims d, const int8_t* __restrict__ S8, const int32_t* __
         for (int i = 0; i < kAheadI8; ++i) {
             const int c = c0 + i;
             if (c < d.nc) {
-                *reinterpret_cast<uint4*>(hc + c * stride) = pack();
-                const uint32_t w[4] = {sv[i].x, sv[i].y, sv[i].z, sv[i].w};
+                *reinterpret_cast<uint4*>(hc + c * stride) = hw;        // the state entering chunk c
+                const uint32_t hv[4] = {hw.x, hw.y, hw.z, hw.w}, sw[4] = {sv[i].x, sv[i].y, sv[i].z, sv[i].w};
+                uint32_t out[4];
+                if (shift <= 7 && qv[i] <= (1 << shift)) {
+                    // two codes per 16-bit field pair (decay codes are at most 2^k when A dt <= 0)
+                    const uint32_t k0 = (uint32_t)((1 << (shift - 1)) + 128 * ((1 << shift) - qv[i])) * 0x10001u;
 #pragma unroll
-                for (int v = 0; v < kVecI8; ++v) {
-                    const int sc = (int)(int8_t)(w[v >> 2] >> (8 * (v & 3)));     // sign-extended code
-                    hv[v] = sat127(sc + ((qv[i] * hv[v] + half) >> shift));
+                    for (int j = 0; j < 4; ++j) out[j] = chain_word(hv[j], sw[j], (uint32_t)qv[i], k0, shift, lo, hi);
+                } else {
+                    const int half = 1 << (shift - 1);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        out[j] = 0u;
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int hs = (int)(int8_t)(hv[j] >> (8 * v)), sc = (int)(int8_t)(sw[j] >> (8 * v));
+                            out[j] |= ((uint32_t)sat127(sc + ((qv[i] * hs + half) >> shift)) & 0xffu) << (8 * v);
+                        }
+                    }
                 }
+                hw = make_uint4(out[0], out[1], out[2], out[3]);
             }
         }
     }
-    *reinterpret_cast<uint4*>(final_state + ((long long)b * d.H + h) * PN + e) = pack();
+    *reinterpret_cast<uint4*>(final_state + ((long long)b * d.H + h) * PN + e) = hw;
 }
 
 }  // namespace

@@ -87,6 +87,22 @@ def test_i8_bit_exact_and_within_tolerance(torch_cuda, name):
     assert rel_l2(y, ey) <= TOL_I8_Y, rel_l2(y, ey)
 
 
+@pytest.mark.parametrize("shift", [5, 9])
+def test_i8_other_decay_shifts_bit_exact(torch_cuda, shift):
+    """Decay shift 5 takes StatePassing's two-codes-per-field carry, 9 its code-at-a-time one."""
+    w = CASES["ragged-q256"]
+    inp, pb = _problem(torch_cuda, w)
+    sc = oracle_scales(inp, w.chunk, w.calib_prefix)
+    pb.set_scales(sc["s_B"], sc["s_C"], sc["s_x"], sc["s_s"], shift)
+    dbg = pb.run_i8_debug()
+    torch_cuda.cuda.synchronize()
+    r = oracle_i8(inp, sc, w.chunk, shift)
+    for k in ("dq", "S8", "H8", "acc_scan1"):
+        np.testing.assert_array_equal(host(dbg[k]), r[k], err_msg=k)
+    np.testing.assert_array_equal(host(pb.final8), r["final8"])
+    assert rel_l2(bf16_to_np(pb.y), r["y"]) <= 1e-2
+
+
 def test_i8_production_call_equals_debug_call(torch_cuda):
     w = CASES["ragged-q256"]
     inp, pb = _problem(torch_cuda, w)
