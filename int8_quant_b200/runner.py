@@ -131,6 +131,18 @@ class SsdProblem:
         return dbg
 
 
+def plan_groups(batch: int, seqlen: int, chunk: int, rows_per_group: int = 1, seg_len: int | None = None):
+    """The copy groups of StreamedScan: (first row, rows, first token, tokens) in enqueue order, and the
+    segment length.  Whole rows (seg_len None or >= seqlen) in groups of rows_per_group, or one row's
+    segments of seg_len tokens (a multiple of the chunk), the last one possibly shorter."""
+    seg = seqlen if seg_len is None or seg_len >= seqlen else int(seg_len)
+    if seg < seqlen:
+        assert rows_per_group == 1 and seg % chunk == 0, "segments: one row per group, whole chunks"
+    groups = [(r, min(rows_per_group, batch - r), t0, min(seg, seqlen - t0))
+              for r in range(0, batch, rows_per_group) for t0 in range(0, max(seqlen, 1), max(seg, 1))]
+    return groups, seg
+
+
 class StreamedScan:
     """A batch held in pinned host memory, scanned in groups with the copies overlapped:
     host->device copies, scans and device->host copies run on three streams, groups taking
@@ -152,13 +164,8 @@ class StreamedScan:
         self.h, self.path, self.A, self.D = host, path, A, D
         b, L, H, P = host["x"].shape
         G, N = host["B"].shape[2], host["B"].shape[3]
-        seg = L if seg_len is None or seg_len >= L else int(seg_len)
-        if seg < L:
-            assert rows_per_group == 1 and seg % chunk == 0, "segments: one row per group, whole chunks"
+        self.groups, seg = plan_groups(b, L, chunk, rows_per_group, seg_len)    # (row0, rows, token0, tokens)
         self.rows, self.seg, self.L, self.chunk = rows_per_group, seg, L, chunk
-        # (first row, rows, first token, tokens)
-        self.groups = [(r, min(rows_per_group, b - r), t0, min(seg, L - t0))
-                       for r in range(0, b, rows_per_group) for t0 in range(0, max(L, 1), max(seg, 1))]
         self.shape = ssd.SsdShape.of(rows_per_group, seg, H, P, G, N, chunk)
         dev = torch.device(device)
         i8 = path == "w8a8"
