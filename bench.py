@@ -701,11 +701,17 @@ def main():
     ap.add_argument("--no-storage-variant", action="store_true",
                     help="skip the W8A8 step with the notes' storage variant (FP16 Acs, INT8 CB in HBM)")
     ap.add_argument("--all-configs", action="store_true",
-                    help="also time every other workload on both paths (device time only; adds minutes)")
+                    help="also time every other workload on both paths (device time only); the default on one GPU")
+    ap.add_argument("--no-all-configs", action="store_true", help="time only --workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work per CPU worker")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    # every workload on one GPU by default (input generation dominates its added time); opt-in under torchrun
+    if int(os.environ.get("WORLD_SIZE", "1")) == 1 and args.batch is None and args.seqlen is None:
+        args.all_configs = True
+    if args.no_all_configs:
+        args.all_configs = False
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
