@@ -396,25 +396,38 @@ def run_ours(args, rank, world, dist):
             dist.barrier()
 
     def timed(path, pb=pb):
-        """Step time over the timed loop (CUDA events around all steps, no per-kernel events,
-        so consecutive launches may overlap as they do in use), then the per-kernel split
-        from a second, profiled pass of the same number of steps (an event pair around every
-        kernel)."""
+        """Step time over the timed loop, CUDA events around all its steps.  Inside that loop only
+        the dominant kernel (the largest share of the warm-up steps' device time) is bracketed by
+        an event pair, so its launch time is measured live in the timed region at two events per
+        step; the other kernels' split comes from a profiled pass of the same number of steps
+        right after (an event pair around every kernel adds about 14 us to a W8A8 step)."""
         step = step_fn(path, pb)
+        iq.ssd_profile_filter(None)
+        iq.ssd_profile_reset()
+        iq.ssd_profile_enable(True)
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize()
+        iq.ssd_profile_enable(False)
+        warm = {k: v for k, v in iq.ssd_profile_read().items() if v[1]}
+        dom = max(warm, key=lambda k: warm[k][0])
+        iq.ssd_profile_reset()
+        iq.ssd_profile_filter(dom)
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with ClockSampler(dev) as clk:
             barrier()
             torch.cuda.synchronize()
+            iq.ssd_profile_enable(True)
             ev0.record(stream)
             for _ in range(args.steps):
                 step()
             ev1.record(stream)
             torch.cuda.synchronize()
+            iq.ssd_profile_enable(False)
             barrier()
         ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev) / args.steps
+        dom_t = iq.ssd_profile_read()[dom]
+        iq.ssd_profile_filter(None)
         iq.ssd_profile_reset()
         iq.ssd_profile_enable(True)
         for _ in range(args.steps):
@@ -422,6 +435,7 @@ def run_ours(args, rank, world, dist):
         torch.cuda.synchronize()
         iq.ssd_profile_enable(False)
         kern = iq.ssd_profile_read()
+        kern[dom] = dom_t                                   # the dominant kernel as timed in the timed loop
         return ms, kern, clk.summary()
 
     def roofline(path, kern, w=w):

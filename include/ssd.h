@@ -333,6 +333,10 @@ ssd_status ssd_selftest_bounded_wait(long long limit_cycles, int* status, unsign
 ssd_status ssd_profile_enable(int enable);
 ssd_status ssd_profile_read(int capacity, const char** names, double* ms, long long* calls, int* count);
 ssd_status ssd_profile_reset(void);
+/* Restricts the per-kernel timing to the kernel named `name` (the names ssd_profile_read
+ * reports; the string is copied), so that one kernel can be timed inside a loop with two
+ * events per launch; NULL times every kernel again. */
+ssd_status ssd_profile_filter(const char* name);
 
 #ifdef __cplusplus
 }

@@ -155,6 +155,7 @@ std::vector<double> ms;
 std::vector<long long> calls;
 std::vector<Pending> pending;
 std::vector<cudaEvent_t> pool;
+std::string filter;                     // empty: every kernel
 
 cudaEvent_t get_event() {
     if (!pool.empty()) { cudaEvent_t e = pool.back(); pool.pop_back(); return e; }
@@ -177,7 +178,7 @@ struct Scope {
     cudaEvent_t b = nullptr;
     Scope(const char* name, cudaStream_t s) : st(s) {
         std::lock_guard<std::mutex> g(mu);
-        if (!enabled) return;
+        if (!enabled || (!filter.empty() && filter != name)) return;
         k = kernel_id(name);
         cudaEvent_t a = get_event();
         b = get_event();
@@ -580,6 +581,12 @@ ssd_status ssd_profile_read(int capacity, const char** names, double* ms, long l
         if (ms) ms[i] = prof::ms[i];
         if (calls) calls[i] = prof::calls[i];
     }
+    return SSD_OK;
+}
+
+ssd_status ssd_profile_filter(const char* name) {
+    std::lock_guard<std::mutex> g(prof::mu);
+    prof::filter = name ? std::string(name) : std::string();
     return SSD_OK;
 }
 

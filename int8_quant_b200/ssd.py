@@ -22,7 +22,7 @@ EXPORTS = ("ssd_status_string", "ssd_last_cuda_error", "ssd_workspace_bytes", "s
            "ssd_scan_fwd_i8", "ssd_scan_fwd_i8_debug", "ssd_calibrate_workspace_bytes",
            "ssd_calibrate_i8", "ssd_workspace_status", "ssd_profile_enable", "ssd_profile_read",
            "ssd_profile_reset", "ssd_scan_fwd_bf16_static", "ssd_selftest_bounded_wait",
-           "ssd_scan_fwd_bf16_from_state", "ssd_scan_fwd_i8_from_state", "ssd_decode_step_bf16",
+           "ssd_scan_fwd_bf16_from_state", "ssd_scan_fwd_i8_from_state", "ssd_decode_step_bf16", "ssd_profile_filter",
            "ssd_decode_step_i8", "ssd_out_proj_workspace_bytes", "ssd_out_proj_i8", "ssd_out_proj_status",
            "ssd_static_scratch_status")
 
@@ -123,6 +123,8 @@ def _lib():
         lib.ssd_profile_enable.argtypes = [I]
         lib.ssd_profile_reset.restype = I
         lib.ssd_profile_reset.argtypes = []
+        lib.ssd_profile_filter.restype = I
+        lib.ssd_profile_filter.argtypes = [ctypes.c_char_p]
         lib.ssd_profile_read.restype = I
         lib.ssd_profile_read.argtypes = [I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
                                          ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_int)]
@@ -280,6 +282,11 @@ def ssd_profile_enable(enable: bool) -> None:
 
 def ssd_profile_reset() -> None:
     _check("ssd_profile_reset", _lib().ssd_profile_reset())
+
+
+def ssd_profile_filter(name: str | None) -> None:
+    """Time only the kernel `name` while profiling is enabled (None: every kernel)."""
+    _check("ssd_profile_filter", _lib().ssd_profile_filter(name.encode() if name else None))
 
 
 def ssd_profile_read() -> dict:
