@@ -20,6 +20,7 @@ import hashlib
 import json
 import multiprocessing as mp
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -145,14 +146,23 @@ def measured_bf16_tflops() -> float:
 # capture, keyed by kernel name, with the sha1 of the kernel source it was taken on.
 # A kernel whose source changed since reports null.
 NCU_TRAFFIC = {
-    # batch-2 captures scaled x4 to the batch-8 launch (traffic grows with the batch)
+    # batch-2 captures scaled x4 to the batch-8 launch (traffic grows with the batch); src_sha1 is the
+    # code hash (_code_hash) of the kernel's source at the capture
     ("chunk_scan", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (224.51e6 + 123.36e6),
-                                            "src_sha1": "5df65d9c3ddcc165c290359db6a0362234866ff9"},
+                                            "src_sha1": "acb43f60bf2fbd5eb0e9707b62df12477c28a626"},
     ("chunk_scan", "bf16", "mamba2-2.7b"): {"bytes_per_launch": 4 * (270.60e6 + 128.16e6),
-                                            "src_sha1": "5df65d9c3ddcc165c290359db6a0362234866ff9"},
+                                            "src_sha1": "acb43f60bf2fbd5eb0e9707b62df12477c28a626"},
     ("ssd_fused_i8", "w8a8", "mamba2-2.7b"): {"bytes_per_launch": 4 * (178.17e6 + 176.30e6),
-                                              "src_sha1": "3a08a823dcfb46ab30d6bebff0bd7ab1e004d1e8"},
+                                              "src_sha1": "1fdea2cb386fcb644dba6640df7309df1be58d3c"},
 }
+
+
+def _code_hash(text: str) -> str:
+    """sha1 of a CUDA source with its comments and whitespace removed, so that a capture stays
+    attached to a kernel whose code has not changed."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return hashlib.sha1(re.sub(r"\s+", "", text).encode()).hexdigest()
 
 
 def _src_hash(kernel: str):
@@ -160,8 +170,8 @@ def _src_hash(kernel: str):
          "chunk_cumsum": "cumsum.cu", "quantize_inputs": "quantize.cu", "ssd_fused_i8": "fused_i8.cu"}.get(kernel)
     if not f:
         return None
-    with open(os.path.join(ROOT, "int8_quant_b200", "csrc", f), "rb") as fh:
-        return hashlib.sha1(fh.read()).hexdigest()
+    with open(os.path.join(ROOT, "int8_quant_b200", "csrc", f)) as fh:
+        return _code_hash(fh.read())
 
 
 def traffic_for(kernel: str, path: str, workload: str):

@@ -9,12 +9,15 @@
 // dequantised with s_C s_s[h,p]; LUT_Scan2 = s_C s_B exp(Acs_j - Acs_i) dt_i folds
 // CB's dequantisation into the ChunkScan2 matrix, which runs in bf16 (kind::f16).
 //
-// One CTA per (chunk, batch row, block of up to 8 heads of one group); B and C are
+// One CTA per (chunk, batch row, block of heads of one group; the block size comes from
+// the caller's wave-count model, 20 heads at the Mamba-2 2.7B shape); B and C are
 // shared by the block, so CB is computed once and kept in TMEM, packed to bf16
 // pairs, for all heads.  The work is split over warp roles that run concurrently
 // and hand off through mbarriers:
 //   warp 0      TMA producer: per head the decay rows (Acs, dt), the state tile and
-//               the x tile (double-buffered), plus C and B once.
+//               the x tile (two stages in bf16, three in W8A8, whose shared memory
+//               has room: two heads' loads in flight ahead of the MMAs), plus C and B
+//               once.
 //   warp 1      TMEM allocation and the single MMA-issuing thread: CB; per head
 //               y = C H^T into one of two TMEM accumulator slots (issued as soon as
 //               the slot is free, ahead of the previous head's remaining work, since
@@ -34,6 +37,12 @@
 //               not coalesce).
 // Every wait is bounded; an expired wait raises a shared abort flag that ends all
 // roles, records SSD_ERR_TIMEOUT in the status word, and the CTA frees TMEM.
+//
+// The notes' storage variant (W8A8, chunk 256): with kCB8 the CTA loads the INT8 CB
+// codes that chunk_bmm.cu wrote (one step per tile, folded into the decay vectors)
+// into the B tile's space instead of forming CB, and the builders widen them to bf16;
+// with acs_half the Acs rows arrive as IEEE half and are widened when the decay
+// vectors are formed.
 #include <cuda_fp16.h>
 
 #include "kernels.h"
